@@ -1,0 +1,491 @@
+"""Benchmark: paged decode attention effective KV GB/s and % of B200 HBM peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--block-size B]
+                    [--partition-tokens P] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch: the copy-on-write
+block copies of the step (workloads that share blocks), the append of each
+sequence's new K/V row, then paged decode attention over every sequence's
+context (which includes the new token).  The default workload is the batch-256
+OPT-13B decode layer (40 heads x 128, bf16 KV, contexts uniform in [1, 2048],
+block size 16).  The K/V pool is resident in HBM before the timed region starts
+and is 43x larger than L2, so no L2 flush is needed between steps.
+
+Multi-GPU: one process per GPU (torchrun); the path shards by sequence with no
+exchange, so every rank runs its own replica of the workload and the job's
+throughput is the sum of all ranks' bytes over the slowest rank's time.
+
+`--impl reference` times the CPU oracle (float64 NumPy) on bounded samples of the
+same workload instead; it is the only other place this script runs the oracle.
+"""
+
+import argparse
+import json
+import math
+import multiprocessing as mp
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention effective KV GB/s and % of B200 HBM peak"
+FALLBACK_HBM_GBS = 6650.0
+WORKLOADS = ("opt13b", "llama7b", "cow", "longctx", "tiny")
+DEFAULT_STEPS = {"opt13b": 500, "llama7b": 2000, "cow": 1000, "longctx": 500, "tiny": 200}
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", choices=WORKLOADS, default="opt13b")
+    ap.add_argument("--block-size", type=int, default=16)
+    ap.add_argument("--partition-tokens", type=int, default=None,
+                    help="split-context partition size (default: the workload's, else the library's choice)")
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline time budget")
+    a = ap.parse_args()
+    if a.steps is None:
+        a.steps = DEFAULT_STEPS[a.workload]
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return a
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def job_throughput(bytes_per_step_per_rank, ms_per_step_by_rank):
+    """Whole-job GB/s of independent replicas: all ranks' bytes over the slowest rank's time."""
+    world = len(ms_per_step_by_rank)
+    slowest = max(ms_per_step_by_rank)
+    return bytes_per_step_per_rank * world / (slowest * 1e-3) / 1e9, slowest
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise max of a list of floats over all ranks (the timing rule for N > 1)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline).  Worker processes are
+# forked before this process touches CUDA, and never touch CUDA themselves.
+# ---------------------------------------------------------------------------
+_SAMPLE = None
+
+
+def _cpu_worker_init():
+    # one BLAS thread per worker process: cores used = number of processes
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except ImportError:
+        pass
+
+
+def _oracle_task(i):
+    import oracle
+    c = _SAMPLE["cases"][i]
+    t0 = time.perf_counter()
+    oracle.paged_decode(c["q"], c["k"], c["v"], c["table"], c["ctx"], _SAMPLE["scale"], _SAMPLE["B"],
+                        _SAMPLE["dtype"])
+    return i, time.perf_counter() - t0
+
+
+def make_cpu_sample(wname, block_size, n_seq, seed=7):
+    """Bounded sample of the workload: its first ``n_seq`` context lengths and head
+    geometry, with N(0,1) values placed through a random block table."""
+    from paged_kv_cache_328_b200 import workloads as wl
+    shapes = {"opt13b": (40, 128, "bf16", wl.opt13b_lengths()),
+              "llama7b": (32, 128, "f16", wl.lognormal_lengths(64, wl.BASE_SEED + 2)),
+              "cow": (40, 128, "f16", None), "longctx": (40, 128, "f16", wl.uniform_lengths(8, wl.BASE_SEED + 5,
+                                                                                         16384, 32768)),
+              "tiny": (2, 64, "f32", wl.tiny_lengths())}
+    H, D, dtype, ctx = shapes[wname]
+    if ctx is None:
+        rng = np.random.default_rng(wl.BASE_SEED + 4)
+        ctx = 512 + rng.integers(1, 257, size=128) + 1
+    B = block_size if wname == "opt13b" else (16 if wname != "tiny" else 16)
+    rng = np.random.default_rng(seed)
+    cases = []
+    for c in [int(x) for x in ctx[:n_seq]]:
+        nblk = max(1, -(-c // B))
+        nb = nblk + 2
+        table = rng.permutation(nb)[:nblk].reshape(1, -1)
+        if dtype == "f32":
+            k = rng.standard_normal((nb, H, B, D), dtype=np.float32)
+            v = rng.standard_normal((nb, H, B, D), dtype=np.float32)
+            q = rng.standard_normal((1, H, D), dtype=np.float32)
+        else:
+            k = rng.integers(0, 1 << 16, size=(nb, H, B, D), dtype=np.uint16) & np.uint16(0xBFFF)
+            v = rng.integers(0, 1 << 16, size=(nb, H, B, D), dtype=np.uint16) & np.uint16(0xBFFF)
+            q = rng.integers(0, 1 << 16, size=(1, H, D), dtype=np.uint16) & np.uint16(0xBFFF)
+            if dtype == "f16":  # keep magnitudes moderate: exponent field <= 15
+                k, v, q = (x & np.uint16(0xBBFF) for x in (k, v, q))
+        cases.append(dict(q=q, k=k, v=v, table=table, ctx=np.array([c]), nbytes=c * H * D * (2 if dtype != "f32"
+                                                                                              else 4) * 2))
+    return dict(cases=cases, scale=1.0 / math.sqrt(D), B=B, dtype=dtype, H=H, D=D)
+
+
+def start_cpu_pool(sample):
+    global _SAMPLE
+    _SAMPLE = sample
+    cores = os.cpu_count() or 1
+    ctx = mp.get_context("fork")
+    return ctx.Pool(cores, initializer=_cpu_worker_init), cores
+
+
+def time_oracle(pool, sample, budget_s):
+    """Run the oracle over the sample's sequences (repeating passes) until budget_s elapsed."""
+    n = len(sample["cases"])
+    done_bytes = 0
+    tokens = 0
+    t0 = time.perf_counter()
+    passes = 0
+    while True:
+        for i, _ in pool.imap_unordered(_oracle_task, range(n)):
+            done_bytes += sample["cases"][i]["nbytes"]
+            tokens += int(sample["cases"][i]["ctx"][0])
+        passes += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    wall = time.perf_counter() - t0
+    return done_bytes, tokens, wall, passes
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.lines = []
+        self.proc = None
+        self.t_start = self.t_stop = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.perf_counter(), line.strip()))
+
+    def mark(self, start):
+        if start:
+            self.t_start = time.perf_counter()
+        else:
+            self.t_stop = time.perf_counter()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        inside = [l for t, l in self.lines if self.t_start <= t <= self.t_stop + 0.15]
+        window = "timed region"
+        if not inside:  # timed region shorter than the sampling period: nearest samples
+            inside = [l for t, l in self.lines if self.t_start - 0.3 <= t <= self.t_stop + 0.3]
+            window = "timed region +-0.3 s"
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for l in inside:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm), "window": window}
+
+
+# ---------------------------------------------------------------------------
+# The GPU arm
+# ---------------------------------------------------------------------------
+def traffic_record(workload_key):
+    """dram bytes per decode launch from a committed ncu capture, if the kernel sources are unchanged."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path)).get(workload_key)
+    except (OSError, ValueError):
+        return None
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.join(ROOT, "paged_kv_cache_328_b200", "csrc"))):
+        h.update(open(os.path.join(ROOT, "paged_kv_cache_328_b200", "csrc", f), "rb").read())
+    return rec["dram_bytes_per_launch"] if rec.get("csrc_sha256") == h.hexdigest() else None
+
+
+def run_gpu(a, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import paged_kv_cache_328_b200 as pkv
+    from paged_kv_cache_328_b200 import workloads as wl
+
+    sample = pool = None
+    cores = 0
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        sample = make_cpu_sample(a.workload, a.block_size, n_seq=32 if a.workload != "longctx" else 2)
+        pool, cores = start_cpu_pool(sample)  # forked before any CUDA call
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    pkv.load()
+
+    w = wl.make(a.workload, device=dev, B=a.block_size if a.workload == "opt13b" else None)
+    pt = w.partition_tokens if a.partition_tokens is None else a.partition_tokens
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    ctx = torch.from_numpy(w.context_lens).to(dev)
+    slots = torch.from_numpy(w.slot_mapping).to(dev)
+    pairs = torch.from_numpy(w.cow_pairs.reshape(-1, 2)).to(dev)
+    out = torch.empty((w.S, w.H, w.D), dtype=torch.float32, device=dev)
+    ws = pkv.alloc_workspace(w.q, w.k_pool, bt, pt)
+    split = pkv.partition_tokens(w.S, w.H, w.D, w.B, w.max_blocks, pt) < w.max_blocks * w.B
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = (1 if len(w.cow_pairs) else 0) + 1 + 2 + (1 if split else 0)
+
+    def step(dec_events=None):
+        if len(w.cow_pairs):
+            pkv.kv_block_copy(w.k_pool, w.v_pool, pairs)
+        pkv.kv_cache_append(w.k_new, w.v_new, w.k_pool, w.v_pool, slots)
+        if dec_events is not None:
+            dec_events[0].record(stream)
+        pkv.paged_attn_decode(w.q, w.k_pool, w.v_pool, bt, ctx, w.scale, out=out, partition_tokens=pt,
+                              workspace=ws)
+        if dec_events is not None:
+            dec_events[1].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+    code, reason = pkv.get_device_error(dev)
+    if code != 0:
+        raise RuntimeError(f"device error word after warm-up: {code} reason {reason}")
+
+    clocks = ClockSampler(local_rank)
+    time.sleep(0.3)
+    dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.mark(True)
+    t_start.record(stream)
+    for i in range(a.steps):
+        step(dec[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(False)
+    barrier()
+    ms = t_start.elapsed_time(t_end)
+    dec_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in dec)
+    clk = clocks.summary()
+    if world > 1:
+        ms, dec_ms = max_over_ranks([ms, dec_ms], dist, dev)
+    code, reason = pkv.get_device_error(dev)
+    if code != 0:
+        raise RuntimeError(f"device error word after the timed steps: {code} reason {reason}")
+
+    # ---- end to end through the public API with host buffers ---------------
+    pin = dict(q=w.q.cpu().pin_memory(), k=w.k_new.cpu().pin_memory(), v=w.v_new.cpu().pin_memory(),
+               bt=bt.cpu().pin_memory(), ctx=ctx.cpu().pin_memory(), slots=slots.cpu().pin_memory(),
+               pairs=pairs.cpu().pin_memory())
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(w.q), torch.empty_like(w.k_new), torch.empty_like(w.v_new)
+    dbt, dctx, dsl, dpr = (torch.empty_like(x) for x in (bt, ctx, slots, pairs))
+    h2d = sum(x.numel() * x.element_size() for x in pin.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        dq.copy_(pin["q"], non_blocking=True)
+        dk.copy_(pin["k"], non_blocking=True)
+        dv.copy_(pin["v"], non_blocking=True)
+        dbt.copy_(pin["bt"], non_blocking=True)
+        dctx.copy_(pin["ctx"], non_blocking=True)
+        dsl.copy_(pin["slots"], non_blocking=True)
+        dpr.copy_(pin["pairs"], non_blocking=True)
+        if len(w.cow_pairs):
+            pkv.kv_block_copy(w.k_pool, w.v_pool, dpr)
+        pkv.kv_cache_append(dk, dv, w.k_pool, w.v_pool, dsl)
+        pkv.paged_attn_decode(dq, w.k_pool, w.v_pool, dbt, dctx, w.scale, out=out, partition_tokens=pt,
+                              workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(a.warmup):
+        e2e_step()
+    e_steps = max(3, a.steps // 2)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    if world > 1:
+        e2e_ms = max_over_ranks([e2e_ms], dist, dev)[0]
+
+    kv_bytes = w.kv_bytes_attended()
+    ms_step = ms / a.steps
+    value, _ = job_throughput(kv_bytes, [ms_step] * world)
+    peak, peak_src = measured_peaks()
+    achieved = kv_bytes / (dec_ms * 1e-3) / 1e9
+    wkey = f"{w.name}" + (f"_pt{pt}" if pt else "")
+    result = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": a.steps,
+        "warmup": a.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "num_seqs": w.S, "num_heads": w.H, "head_dim": w.D, "block_size": w.B,
+            "context_tokens_per_step": int(w.context_lens.sum()), "kv_bytes_per_step": kv_bytes,
+            "cow_pairs_per_step": int(len(w.cow_pairs)), "appended_tokens_per_step": int((w.slot_mapping >= 0).sum()),
+            "partition_tokens": pkv.partition_tokens(w.S, w.H, w.D, w.B, w.max_blocks, pt),
+            "l2": f"no flush: K/V pool {w.k_pool.numel() * w.k_pool.element_size() * 2 / 1e9:.2f} GB "
+                  f"= {w.k_pool.numel() * w.k_pool.element_size() * 2 / 126e6:.0f}x L2",
+            "parallelism": f"replicas x{world}",
+        },
+        "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
+        "seq_per_s": round(w.S * world / (ms_step * 1e-3), 1),
+        "ctx_tokens_per_s": round(int(w.context_lens.sum()) * world / (ms_step * 1e-3), 1),
+        "roofline": {
+            "kernel": "paged_attn_decode call (plan + persistent decode + merge launches)",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_source": peak_src,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic_record(wkey),
+            "algorithmic_bytes_per_launch": kv_bytes,
+            "avg_launch_ms": round(dec_ms, 5),
+        },
+        "e2e": {"value": round(kv_bytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5),
+                "note": "per-step inputs (q, new K/V rows, tables, lengths, slots, pairs) copied from pinned "
+                        "host memory and the fp32 output read back; the K/V cache stays resident"},
+        "gpu_launches": launches_per_step * a.steps,
+        "clocks": clk,
+    }
+    if w.name == "cow":
+        result["config"]["cow_memory_saving"] = round(w.info["cow_saving"], 4)
+    result["config"]["last_block_waste"] = round(wl.last_block_waste(w), 4)
+
+    if pool is not None:
+        nbytes, tokens, wall, passes = time_oracle(pool, sample, a.cpu_seconds)
+        pool.terminate()
+        result["cpu_baseline"] = {
+            "value": round(nbytes / wall / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(sample['cases'])} sequences x {sample['H']} heads of the workload's context lengths "
+                      f"({passes} pass(es), {tokens} context tokens per head, {wall:.1f} s), float64 NumPy, "
+                      f"one process per core",
+        }
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# Reference arm: the CPU oracle on bounded samples of the same workload
+# ---------------------------------------------------------------------------
+def run_reference(a, rank, world):
+    if rank != 0:
+        return
+    n_seq = {"opt13b": 4, "llama7b": 16, "cow": 4, "longctx": 1, "tiny": 4}[a.workload]
+    sample = make_cpu_sample(a.workload, a.block_size, n_seq=n_seq)
+    pool, cores = start_cpu_pool(sample)
+    for _ in range(a.warmup):
+        time_oracle(pool, sample, 0.0)
+    step_bytes = sum(c["nbytes"] for c in sample["cases"])
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        time_oracle(pool, sample, 0.0)
+    wall = time.perf_counter() - t0
+    pool.terminate()
+    value = step_bytes * a.steps / wall / 1e9
+    res = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(wall / a.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": a.workload, "block_size": sample["B"], "parallelism": "cpu processes"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n_seq} sequence(s) x {sample['H']} heads per step"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    a = parse()
+    rank, world, local_rank = dist_env()
+    if a.gpus != world and world != 1:
+        print(f"warning: --gpus {a.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if a.impl == "reference":
+        run_reference(a, rank, world)
+        return
+    run_gpu(a, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

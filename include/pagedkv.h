@@ -1,0 +1,211 @@
+/*
+ * pagedkv.h - C ABI of libpagedkv.so: paged single-query decode attention and
+ * the two kernels that maintain a paged KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * What the operations are (sources cited by page title and section):
+ *
+ *  - The KV cache of a sequence is cut into fixed-size blocks of B tokens that
+ *    live anywhere in one shared physical pool; a per-sequence block table maps
+ *    logical block j to its physical block.  Attention follows the table,
+ *    gathers the scattered blocks and computes softmax(Q K^T) V.
+ *    ("PagedAttention - Efficient Memory Management for LLM Serving with vLLM",
+ *    section "Method (PagedAttention + vLLM)"; "LLM Inference 8 - PagedAttention",
+ *    section "PagedAttention", block-table example 0->4, 1->1, 2->7.)
+ *  - Each new token's K and V are stored into the cache and reused by later
+ *    steps; a new block is taken only when the current one is full.
+ *    ("LLM Inference 8 - PagedAttention", sections "KV Cache의 메모리 문제" and
+ *    "PagedAttention의 동작 방식".)
+ *  - Sequences that share a prefix share its physical blocks; when one of them
+ *    writes, only that block is copied (copy-on-write, P3 -> P9 in the
+ *    framework-overview flowchart of the paper digest's "방법 (Method)" section).
+ *
+ * Layout (the pages fix only the logical->physical indirection; this is the
+ * library's choice): K and V are separate pools, each [num_blocks][num_heads]
+ * [block_size][head_dim], row-major, in one storage dtype.  Token t of sequence
+ * s, head h is element (block_tables[s][t / B], h, t % B, :).  One (block, head)
+ * chunk is B * head_dim contiguous elements.
+ *
+ * Conventions for every entry point:
+ *  - All data pointers are DEVICE pointers owned by the caller; the library keeps
+ *    no reference after the call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and never synchronise the host, except pkv_get_device_error.
+ *  - Return 0 (PKV_OK) or a negative PKV_E* code.  Argument checks happen on the
+ *    host before any CUDA call; a rejected call launches nothing and touches no
+ *    memory.
+ *  - Device-side checks (block id outside [0, num_blocks), context length outside
+ *    [0, max_blocks_per_seq * B], slot outside [-1, num_blocks * B), copy pair
+ *    outside the pool, a bounded wait that ran out) skip the offending access
+ *    and set a sticky per-device error word; no kernel traps.  Outputs that
+ *    depend on a flagged access are unspecified.  Read the word with
+ *    pkv_get_device_error.
+ *  - Supported: head_dim in {64, 128}; block_size in {8, 16, 32, 64, 128};
+ *    storage dtype fp32, fp16 or bf16.  q, K, V, new K/V, out and workspace
+ *    pointers must be 16-byte aligned.
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Storage dtype of q, the K/V pools and appended rows. */
+typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+
+/* Return codes. */
+enum {
+  PKV_OK = 0,
+  PKV_EINVAL = -1,        /* a null pointer, a negative or too-large size, bad partition size */
+  PKV_EDTYPE = -2,        /* dtype is not a pkv_dtype */
+  PKV_EALIGN = -3,        /* a pointer is not aligned as required */
+  PKV_EUNSUPPORTED = -4,  /* head_dim or block_size not in the supported set */
+  PKV_ECUDA = -5,         /* a CUDA runtime call or a kernel launch failed */
+  PKV_EWORKSPACE = -6,    /* workspace smaller than paged_attn_decode_workspace_size() */
+  PKV_EDEVICE = -7,       /* a kernel flagged bad device data (see pkv_get_device_error) */
+  PKV_ETIMEOUT = -8       /* a kernel's bounded wait ran out (see pkv_get_device_error) */
+};
+
+/* Reasons stored in the device error word (the `reason` of pkv_get_device_error). */
+enum {
+  PKV_DEV_OK = 0,
+  PKV_DEV_BLOCK_ID = 1,     /* a block-table entry outside [0, num_blocks) was needed */
+  PKV_DEV_CONTEXT_LEN = 2,  /* a context length outside [0, max_blocks_per_seq * B] */
+  PKV_DEV_SLOT = 3,         /* an append slot >= num_blocks * B */
+  PKV_DEV_COPY_PAIR = 4,    /* a copy pair with a block id outside [0, num_blocks) */
+  PKV_DEV_WAIT_TIMEOUT = 5  /* a shared-memory pipeline wait exceeded its bound */
+};
+
+/*
+ * paged_attn_decode - one query token per sequence attends over its paged context.
+ *
+ * For every sequence s < num_seqs and head h < num_heads:
+ *   out[s][h][:] = sum_t w_t * V_t,  w = softmax_t(scale * <q[s][h], K_t>),
+ * over the context_lens[s] tokens t reached through block_tables[s]
+ * ("PagedAttention - Efficient Memory Management for LLM Serving with vLLM",
+ * section "Method (PagedAttention + vLLM)").  A context of length 0 gives out = 0.
+ *
+ *   q             [num_seqs][num_heads][head_dim], storage dtype.
+ *   k_cache,
+ *   v_cache       [num_blocks][num_heads][block_size][head_dim], storage dtype.
+ *   block_tables  int32 [num_seqs][max_blocks_per_seq]; entries past a sequence's
+ *                 last block are never read (pad with -1).
+ *   context_lens  int32 [num_seqs], 0 <= ctx <= max_blocks_per_seq * block_size.
+ *   scale         multiplies q.k before the softmax (typically 1/sqrt(head_dim)).
+ *   out           float32 [num_seqs][num_heads][head_dim].
+ *   partition_tokens  split-context partition size in tokens: 0 = library choice;
+ *                 otherwise a positive multiple of block_size.  A context longer
+ *                 than one partition is processed as independent partitions whose
+ *                 partial softmax states are merged exactly (log-sum-exp); a
+ *                 partition size >= max_blocks_per_seq * block_size means no split.
+ *   workspace     device scratch of at least paged_attn_decode_workspace_size()
+ *                 bytes, 16-byte aligned.  It holds the call's work list (a few
+ *                 bytes per sequence) and, when the call splits, the partitions'
+ *                 partial softmax states.  Contents on entry do not matter; calls
+ *                 that share one workspace must be ordered on one stream.  If NULL,
+ *                 the library takes it from the stream-ordered allocator
+ *                 (cudaMallocAsync / cudaFreeAsync on `stream`).
+ *   stream        cudaStream_t.
+ */
+int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, const int32_t* context_lens,
+                      int num_seqs, int num_heads, int head_dim, int block_size,
+                      int max_blocks_per_seq, int num_blocks, pkv_dtype dtype,
+                      float scale, float* out, int partition_tokens,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace bytes paged_attn_decode needs for these sizes and partition_tokens
+ * (0 = the library's choice, resolved exactly as paged_attn_decode resolves it):
+ * 16 + 4 * num_seqs * P rounded up to 16, plus 8 * S * H * P and 4 * S * H * P *
+ * head_dim (each rounded up to 16) when the call splits into P > 1 partitions.
+ * Returns (size_t)-1 for arguments paged_attn_decode would reject.  Pure host
+ * function.
+ */
+size_t paged_attn_decode_workspace_size(int num_seqs, int num_heads, int head_dim,
+                                        int block_size, int max_blocks_per_seq,
+                                        int partition_tokens);
+
+/*
+ * The partition size paged_attn_decode will use for these arguments (resolving
+ * partition_tokens = 0), or a negative PKV_E* code.  Pure host function.
+ */
+int paged_attn_decode_partition_tokens(int num_seqs, int num_heads, int head_dim,
+                                       int block_size, int max_blocks_per_seq,
+                                       int partition_tokens);
+
+/*
+ * kv_cache_append - store the step's new K and V rows into their cache slots.
+ *
+ * For every token t < num_tokens with slot = slot_mapping[t] >= 0:
+ *   k_cache[slot / B][h][slot % B][:] = k[t][h][:]   (and the same for v), all h.
+ * ("LLM Inference 8 - PagedAttention", section "KV Cache의 메모리 문제": the new
+ * token's Key and Value are added to the cache.)  slot = -1 skips the token; a
+ * slot >= num_blocks * B is skipped and flagged (PKV_DEV_SLOT).  Two tokens
+ * with the same slot race (unspecified which one lands).  Bit-exact copy.
+ *
+ *   k, v          [num_tokens][num_heads][head_dim], storage dtype.
+ *   slot_mapping  int64 [num_tokens].
+ */
+int kv_cache_append(const void* k, const void* v, void* k_cache, void* v_cache,
+                    const int64_t* slot_mapping, int num_tokens, int num_heads,
+                    int head_dim, int block_size, int num_blocks, pkv_dtype dtype,
+                    void* stream);
+
+/*
+ * kv_block_copy - copy-on-write block copies.
+ *
+ * For every pair i < num_pairs, (src, dst) = (src_dst_pairs[2i], src_dst_pairs[2i+1]):
+ *   k_cache[dst] = k_cache[src] and v_cache[dst] = v_cache[src]
+ * (all heads, all block_size slots).  ("PagedAttention - Efficient Memory
+ * Management for LLM Serving with vLLM", section "Method (PagedAttention +
+ * vLLM)", copy-on-write: only the written block is copied.)  Pairs must not
+ * overlap: no dst may repeat or appear as any src, and src != dst; overlapping
+ * pairs race.  A pair with an id outside [0, num_blocks) is skipped and flagged
+ * (PKV_DEV_COPY_PAIR).  Bit-exact copy.
+ *
+ *   src_dst_pairs int64 [num_pairs][2], device memory.
+ */
+int kv_block_copy(void* k_cache, void* v_cache, const int64_t* src_dst_pairs,
+                  int num_pairs, int num_heads, int head_dim, int block_size,
+                  int num_blocks, pkv_dtype dtype, void* stream);
+
+/*
+ * paged_kv_gather - copy one sequence's cached rows into contiguous memory.
+ *
+ * out[h][t][:] = cache[block_table_row[t / B]][h][t % B][:] for t < context_len,
+ * bit for bit, through the same address computation the decode kernel uses.
+ * For checking block-table indexing and for exporting a sequence.
+ *
+ *   cache            one pool, [num_blocks][num_heads][block_size][head_dim].
+ *   block_table_row  int32 [>= ceil(context_len / block_size)], device memory.
+ *   context_len      host int, >= 0.
+ *   out              [num_heads][context_len][head_dim], storage dtype.
+ */
+int paged_kv_gather(const void* cache, const int32_t* block_table_row, int context_len,
+                    int num_heads, int head_dim, int block_size, int num_blocks,
+                    pkv_dtype dtype, void* out, void* stream);
+
+/*
+ * pkv_get_device_error - synchronise `stream`, read and clear the device error
+ * word of the current device.  Returns PKV_OK when it was clear, PKV_ETIMEOUT when
+ * it records PKV_DEV_WAIT_TIMEOUT, PKV_EDEVICE for any other reason, PKV_ECUDA if
+ * the synchronisation or the read failed.  *reason (may be NULL) receives the
+ * first PKV_DEV_* reason recorded since the last clear.
+ */
+int pkv_get_device_error(void* stream, int* reason);
+
+/* Static description of a return code. */
+const char* pkv_strerror(int code);
+
+/* ABI version of this header (incremented on incompatible changes). */
+int pkv_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H_ */

@@ -1,0 +1,216 @@
+"""ctypes binding of libpagedkv.so (the C ABI in include/pagedkv.h).
+
+Argument marshalling only: every function checks that the tensors are CUDA,
+contiguous and of the expected dtypes, passes their device pointers and the
+current torch stream to the C entry point of the same name, and raises
+``PagedKVError`` on a non-zero return.  There is no fallback: if the shared
+library is missing, or a tensor is not on a CUDA device, the call fails.
+"""
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedkv.so")
+
+PKV_F32, PKV_F16, PKV_BF16 = 0, 1, 2
+DTYPE_CODE = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16}
+
+ERRORS = {
+    0: "PKV_OK", -1: "PKV_EINVAL", -2: "PKV_EDTYPE", -3: "PKV_EALIGN", -4: "PKV_EUNSUPPORTED",
+    -5: "PKV_ECUDA", -6: "PKV_EWORKSPACE", -7: "PKV_EDEVICE", -8: "PKV_ETIMEOUT",
+}
+DEVICE_REASONS = {0: "ok", 1: "block id", 2: "context length", 3: "slot", 4: "copy pair", 5: "wait timeout"}
+
+# Every symbol the header declares, with its ctypes signature.
+_c_void_p, _c_int, _c_float, _c_size_t = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "paged_attn_decode": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                   _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                   _c_float, _c_void_p, _c_int, _c_void_p, _c_size_t, _c_void_p]),
+    "paged_attn_decode_workspace_size": (_c_size_t, [_c_int] * 6),
+    "paged_attn_decode_partition_tokens": (_c_int, [_c_int] * 6),
+    "kv_cache_append": (_c_int, [_c_void_p] * 5 + [_c_int] * 6 + [_c_void_p]),
+    "kv_block_copy": (_c_int, [_c_void_p] * 3 + [_c_int] * 6 + [_c_void_p]),
+    "paged_kv_gather": (_c_int, [_c_void_p, _c_void_p] + [_c_int] * 6 + [_c_void_p, _c_void_p]),
+    "pkv_get_device_error": (_c_int, [_c_void_p, ctypes.POINTER(_c_int)]),
+    "pkv_strerror": (ctypes.c_char_p, [_c_int]),
+    "pkv_abi_version": (_c_int, []),
+}
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        msg = f"{where}: {ERRORS.get(code, code)} ({strerror(code) if _LIB else code})"
+        super().__init__(msg)
+
+
+_LIB = None
+
+
+def load(path=LIB_PATH):
+    """Load the shared library (once) and declare every entry point's signature."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is not built: run `python -m paged_kv_cache_328_b200.build` "
+                "(nvcc, sm_100a). There is no CPU fallback.")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def strerror(code):
+    return load().pkv_strerror(code).decode()
+
+
+def abi_version():
+    return load().pkv_abi_version()
+
+
+def _check(rc, where):
+    if rc != 0:
+        raise PagedKVError(rc, where)
+
+
+def _cuda(t, name, dtypes=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device}); there is no CPU path")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    return t.data_ptr()
+
+
+def _stream(device, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def workspace_size(num_seqs, num_heads, head_dim, block_size, max_blocks, partition_tokens=0):
+    n = load().paged_attn_decode_workspace_size(num_seqs, num_heads, head_dim, block_size, max_blocks,
+                                                partition_tokens)
+    if n == ctypes.c_size_t(-1).value:
+        raise PagedKVError(-1, "paged_attn_decode_workspace_size")
+    return n
+
+
+def partition_tokens(num_seqs, num_heads, head_dim, block_size, max_blocks, partition_tokens=0):
+    rc = load().paged_attn_decode_partition_tokens(num_seqs, num_heads, head_dim, block_size, max_blocks,
+                                                   partition_tokens)
+    if rc < 0:
+        raise PagedKVError(rc, "paged_attn_decode_partition_tokens")
+    return rc
+
+
+def alloc_workspace(q, k_cache, block_tables, partition_tokens=0):
+    """A uint8 workspace tensor sized for these inputs, on q's device."""
+    S, H, D = q.shape
+    B = k_cache.shape[2]
+    n = workspace_size(S, H, D, B, block_tables.shape[1], partition_tokens)
+    return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+
+def paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out=None,
+                      partition_tokens=0, workspace=None, stream=None):
+    """out[s, h] = softmax(scale * K q) V over the paged context; returns out (float32 [S, H, D])."""
+    lib = load()
+    S, H, D = q.shape
+    NB, Hc, B, Dc = k_cache.shape
+    if (Hc, Dc) != (H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("q [S,H,D] and caches [NB,H,B,D] disagree")
+    if q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise TypeError("q, k_cache and v_cache must share one storage dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables must be [S, max_blocks] and context_lens [S]")
+    _cuda(q, "q", DTYPE_CODE)
+    if out is None:
+        out = torch.empty((S, H, D), dtype=torch.float32, device=q.device)
+    if out.shape != (S, H, D) or out.dtype != torch.float32:
+        raise ValueError("out must be float32 [S, H, D]")
+    if workspace is None:
+        workspace = alloc_workspace(q, k_cache, block_tables, partition_tokens)
+    dt = DTYPE_CODE[k_cache.dtype]
+    args = (_cuda(q, "q", DTYPE_CODE), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+            _cuda(block_tables, "block_tables", (torch.int32,)),
+            _cuda(context_lens, "context_lens", (torch.int32,)),
+            S, H, D, B, block_tables.shape[1], NB, dt, float(scale),
+            _cuda(out, "out", (torch.float32,)), int(partition_tokens),
+            _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size())
+    with torch.cuda.device(q.device):
+        rc = lib.paged_attn_decode(*args, _stream(q.device, stream))
+    _check(rc, "paged_attn_decode")
+    return out
+
+
+def kv_cache_append(k, v, k_cache, v_cache, slot_mapping, stream=None):
+    """k_cache[slot // B, :, slot % B] = k[t] (and v) for every t with slot >= 0."""
+    lib = load()
+    T, H, D = k.shape
+    NB, Hc, B, Dc = k_cache.shape
+    if (Hc, Dc) != (H, D) or v.shape != k.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("k/v [T,H,D] and caches [NB,H,B,D] disagree")
+    if slot_mapping.shape != (T,):
+        raise ValueError("slot_mapping must be [T]")
+    if k.dtype != k_cache.dtype or v.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise TypeError("new rows and caches must share one storage dtype")
+    args = (_cuda(k, "k", DTYPE_CODE), _cuda(v, "v", DTYPE_CODE), _cuda(k_cache, "k_cache"),
+            _cuda(v_cache, "v_cache"), _cuda(slot_mapping, "slot_mapping", (torch.int64,)),
+            T, H, D, B, NB, DTYPE_CODE[k_cache.dtype])
+    with torch.cuda.device(k_cache.device):
+        rc = lib.kv_cache_append(*args, _stream(k_cache.device, stream))
+    _check(rc, "kv_cache_append")
+
+
+def kv_block_copy(k_cache, v_cache, src_dst_pairs, stream=None):
+    """k_cache[dst] = k_cache[src] and v_cache[dst] = v_cache[src] for each (src, dst) pair."""
+    lib = load()
+    NB, H, B, D = k_cache.shape
+    if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
+        raise ValueError("k_cache and v_cache disagree")
+    if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [n, 2]")
+    args = (_cuda(k_cache, "k_cache", DTYPE_CODE), _cuda(v_cache, "v_cache", DTYPE_CODE),
+            _cuda(src_dst_pairs, "src_dst_pairs", (torch.int64,)), src_dst_pairs.shape[0],
+            H, D, B, NB, DTYPE_CODE[k_cache.dtype])
+    with torch.cuda.device(k_cache.device):
+        rc = lib.kv_block_copy(*args, _stream(k_cache.device, stream))
+    _check(rc, "kv_block_copy")
+
+
+def paged_kv_gather(cache, block_table_row, context_len, out=None, stream=None):
+    """Contiguous [H, context_len, D] copy of one sequence's rows of one pool."""
+    lib = load()
+    NB, H, B, D = cache.shape
+    _cuda(cache, "cache", DTYPE_CODE)
+    if out is None:
+        out = torch.empty((H, context_len, D), dtype=cache.dtype, device=cache.device)
+    if out.shape != (H, context_len, D) or out.dtype != cache.dtype:
+        raise ValueError("out must be [H, context_len, D] in the cache dtype")
+    args = (_cuda(cache, "cache", DTYPE_CODE), _cuda(block_table_row, "block_table_row", (torch.int32,)),
+            int(context_len), H, D, B, NB, DTYPE_CODE[cache.dtype], _cuda(out, "out"))
+    with torch.cuda.device(cache.device):
+        rc = lib.paged_kv_gather(*args, _stream(cache.device, stream))
+    _check(rc, "paged_kv_gather")
+    return out
+
+
+def get_device_error(device=None, stream=None):
+    """Synchronise the stream, read and clear the device error word: (code, reason)."""
+    lib = load()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    reason = ctypes.c_int(0)
+    with torch.cuda.device(dev):
+        rc = lib.pkv_get_device_error(_stream(dev, stream), ctypes.byref(reason))
+    return rc, reason.value

@@ -1,0 +1,97 @@
+// Cache-maintenance kernels: per-token append into slots, copy-on-write block
+// copy, and a contiguous gather of one sequence.  All three are pure data
+// movement in 16-byte vectors; the copies are bit-exact.
+#pragma once
+
+#include "pkv_device.cuh"
+
+namespace pkv {
+
+// kv_cache_append: one thread per 16-byte vector of one (token, K|V, head) row.
+// row_vecs = head_dim * elem_bytes / 16.  Grid-stride over
+// num_tokens * 2 * num_heads * row_vecs vectors.
+__global__ void __launch_bounds__(256)
+    kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, uint4* __restrict__ k_cache,
+                     uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int num_tokens,
+                     int num_heads, int row_vecs, int block_size, long long num_slots) {
+  const long long per_token = 2LL * num_heads * row_vecs;
+  const long long total = (long long)num_tokens * per_token;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(i / per_token);
+    long long r = i - (long long)t * per_token;
+    const int is_v = (int)(r / ((long long)num_heads * row_vecs));
+    r -= (long long)is_v * num_heads * row_vecs;
+    const int h = (int)(r / row_vecs);
+    const int vec = (int)(r - (long long)h * row_vecs);
+    const long long slot = slot_mapping[t];
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (is_v == 0 && h == 0 && vec == 0) flag_error(PKV_DEV_SLOT);
+      continue;
+    }
+    const long long blk = slot / block_size;
+    const long long off = slot - blk * block_size;
+    const size_t dst = pool_row(blk, h, off, num_heads, block_size, row_vecs) + vec;
+    const size_t src = ((size_t)t * num_heads + h) * row_vecs + vec;
+    if (is_v)
+      v_cache[dst] = v_new[src];
+    else
+      k_cache[dst] = k_new[src];
+  }
+}
+
+// kv_block_copy: grid = (chunks per block, num_pairs, 2 for K|V); each thread moves
+// kCopyVecs 16-byte vectors, all loads issued before the stores.
+constexpr int kCopyThreads = 256;
+constexpr int kCopyVecs = 4;
+
+__global__ void __launch_bounds__(kCopyThreads)
+    kv_block_copy_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                         const int64_t* __restrict__ pairs, long long block_vecs, int num_blocks) {
+  const long long src = pairs[2 * (size_t)blockIdx.y];
+  const long long dst = pairs[2 * (size_t)blockIdx.y + 1];
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (blockIdx.x == 0 && blockIdx.z == 0 && threadIdx.x == 0) flag_error(PKV_DEV_COPY_PAIR);
+    return;
+  }
+  uint4* pool = blockIdx.z ? v_cache : k_cache;
+  const uint4* from = pool + (size_t)src * block_vecs;
+  uint4* to = pool + (size_t)dst * block_vecs;
+  const long long base = (long long)blockIdx.x * (kCopyThreads * kCopyVecs) + threadIdx.x;
+  uint4 buf[kCopyVecs];
+#pragma unroll
+  for (int j = 0; j < kCopyVecs; ++j) {
+    const long long idx = base + (long long)j * kCopyThreads;
+    if (idx < block_vecs) buf[j] = from[idx];
+  }
+#pragma unroll
+  for (int j = 0; j < kCopyVecs; ++j) {
+    const long long idx = base + (long long)j * kCopyThreads;
+    if (idx < block_vecs) to[idx] = buf[j];
+  }
+}
+
+// paged_kv_gather: out[h][t][:] = cache[table[t / B]][h][t % B][:].  Rows are
+// addressed with pool_row, the helper the decode kernel's producer uses.
+__global__ void __launch_bounds__(256)
+    kv_gather_kernel(const uint4* __restrict__ cache, const int32_t* __restrict__ table, int context_len,
+                     int num_heads, int row_vecs, int block_size, int num_blocks, uint4* __restrict__ out) {
+  const long long total = (long long)num_heads * context_len * row_vecs;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int h = (int)(i / ((long long)context_len * row_vecs));
+    long long r = i - (long long)h * context_len * row_vecs;
+    const int t = (int)(r / row_vecs);
+    const int vec = (int)(r - (long long)t * row_vecs);
+    const int phys = table[t / block_size];
+    if (phys < 0 || phys >= num_blocks) {
+      if (vec == 0) flag_error(PKV_DEV_BLOCK_ID);
+      continue;
+    }
+    const size_t src = pool_row(phys, h, t % block_size, num_heads, block_size, row_vecs) + vec;
+    out[i] = cache[src];
+  }
+}
+
+}  // namespace pkv

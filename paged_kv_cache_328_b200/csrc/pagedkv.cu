@@ -1,0 +1,353 @@
+// libpagedkv: the C ABI declared in include/pagedkv.h.
+//
+// Host side only: argument validation (before any CUDA call), resolution of the
+// split-context partition size, workspace layout, and kernel launches.  The
+// kernels live in decode.cuh (paged decode attention: plan, persistent decode,
+// log-sum-exp merge) and cache_ops.cuh (append, block copy, gather).
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "pagedkv.h"
+#include "pkv_device.cuh"
+#include "decode.cuh"
+#include "cache_ops.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int elem_bytes(pkv_dtype dt) {
+  switch (dt) {
+    case PKV_F32: return 4;
+    case PKV_F16: return 2;
+    case PKV_BF16: return 2;
+  }
+  return 0;
+}
+
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+bool block_size_ok(int b) { return b == 8 || b == 16 || b == 32 || b == 64 || b == 128; }
+
+size_t round16(size_t x) { return (x + 15) / 16 * 16; }
+
+// ---------------------------------------------------------------------------
+// Decode plan: partition size and workspace layout.
+// ---------------------------------------------------------------------------
+struct DecodePlan {
+  int part_tokens = 0;
+  int max_parts = 1;
+  bool split = false;
+  size_t off_units = 0, off_ml = 0, off_acc = 0, bytes = 0;
+};
+
+// Library choice of partition size when the caller passes 0: contexts longer than
+// 512 tokens are split into 512-token partitions (a multiple of every supported
+// block size), which bounds the work of one unit so that the persistent CTAs
+// finish together; shorter maximum contexts are not split.
+constexpr int kAutoPartitionTokens = 512;
+
+int make_plan(int S, int H, int D, int B, int MB, int requested, DecodePlan* plan) {
+  if (S < 0 || H <= 0 || MB <= 0) return PKV_EINVAL;
+  if (!head_dim_ok(D) || !block_size_ok(B)) return PKV_EUNSUPPORTED;
+  if (S > 65535 || H > 65535) return PKV_EINVAL;
+  const long long max_ctx = (long long)MB * B;
+  if (max_ctx > (INT_MAX / 2)) return PKV_EINVAL;
+  if (requested < 0 || (requested > 0 && requested % B != 0)) return PKV_EINVAL;
+  long long pt = requested > 0 ? requested : kAutoPartitionTokens;
+  if (pt >= max_ctx) pt = max_ctx;
+  const long long parts = (max_ctx + pt - 1) / pt;
+  if (parts > 32767) return PKV_EINVAL;
+  if ((long long)S * H * parts > (long long)INT_MAX / 2) return PKV_EINVAL;
+  plan->part_tokens = (int)pt;
+  plan->max_parts = (int)parts;
+  plan->split = parts > 1;
+  size_t off = 16;  // counters[2] (+ padding)
+  plan->off_units = off;
+  off += round16((size_t)S * parts * sizeof(uint32_t));
+  if (plan->split) {
+    plan->off_ml = off;
+    off += round16((size_t)S * H * parts * sizeof(float2));
+    plan->off_acc = off;
+    off += round16((size_t)S * H * parts * D * sizeof(float));
+  }
+  plan->bytes = off;
+  return PKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Per-device launch facts, filled on first use.
+// ---------------------------------------------------------------------------
+std::mutex g_mu;
+int g_sm_count[kMaxDevices];
+
+int current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return PKV_ECUDA;
+  return PKV_OK;
+}
+
+int sm_count(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 0;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+// Resident CTAs per SM of one decode instantiation (after raising its shared-memory limit).
+template <typename T, int D, int TT, int NS>
+int decode_occupancy(int dev) {
+  static int occ[kMaxDevices];
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (occ[dev] == 0) {
+    using Tr = pkv::DecodeTraits<T, D, TT, NS>;
+    auto kern = pkv::paged_decode_kernel<T, D, TT, NS>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::kSmemBytes) != cudaSuccess)
+      return 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, pkv::kDecodeThreads, Tr::kSmemBytes) !=
+            cudaSuccess ||
+        n <= 0)
+      return 0;
+    occ[dev] = n;
+  }
+  return occ[dev];
+}
+
+template <typename T, int D, int TT, int NS>
+int launch_decode(const pkv::DecodeParams& prm, long long max_units, cudaStream_t st) {
+  using Tr = pkv::DecodeTraits<T, D, TT, NS>;
+  int dev;
+  if (current_device(&dev) != PKV_OK) return PKV_ECUDA;
+  const int sms = sm_count(dev);
+  const int occ = decode_occupancy<T, D, TT, NS>(dev);
+  if (sms <= 0 || occ <= 0) return PKV_ECUDA;
+  long long grid = (long long)sms * occ;
+  if (grid > max_units) grid = max_units;
+  if (grid < 1) grid = 1;
+  pkv::paged_decode_kernel<T, D, TT, NS><<<(unsigned)grid, pkv::kDecodeThreads, Tr::kSmemBytes, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+// Tile sizes: every stage holds 32 KB of K+V (64 rows of 256 bytes for 16-bit
+// D=128); three stages per CTA, two CTAs per SM.
+template <int D>
+int dispatch_decode(pkv_dtype dt, const pkv::DecodeParams& prm, long long max_units, cudaStream_t st) {
+  constexpr int kTT16 = 16384 / (D * 2);
+  constexpr int kTT32 = 16384 / (D * 4);
+  switch (dt) {
+    case PKV_F16: return launch_decode<__half, D, kTT16, 3>(prm, max_units, st);
+    case PKV_BF16: return launch_decode<__nv_bfloat16, D, kTT16, 3>(prm, max_units, st);
+    case PKV_F32: return launch_decode<float, D, kTT32, 3>(prm, max_units, st);
+  }
+  return PKV_EDTYPE;
+}
+
+int grid_for(long long work, int per_block, int dev) {
+  long long blocks = (work + per_block - 1) / per_block;
+  const int sms = sm_count(dev);
+  const long long cap = (long long)(sms > 0 ? sms : 148) * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return (int)blocks;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t paged_attn_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int block_size,
+                                        int max_blocks_per_seq, int partition_tokens) {
+  DecodePlan plan;
+  if (make_plan(num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens, &plan) != PKV_OK)
+    return (size_t)-1;
+  return plan.bytes;
+}
+
+int paged_attn_decode_partition_tokens(int num_seqs, int num_heads, int head_dim, int block_size,
+                                       int max_blocks_per_seq, int partition_tokens) {
+  DecodePlan plan;
+  const int rc = make_plan(num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens, &plan);
+  return rc != PKV_OK ? rc : plan.part_tokens;
+}
+
+int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, int num_seqs, int num_heads, int head_dim, int block_size,
+                      int max_blocks_per_seq, int num_blocks, pkv_dtype dtype, float scale, float* out,
+                      int partition_tokens, void* workspace, size_t workspace_bytes, void* stream) {
+  if (elem_bytes(dtype) == 0) return PKV_EDTYPE;
+  DecodePlan plan;
+  const int rc = make_plan(num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens, &plan);
+  if (rc != PKV_OK) return rc;
+  if (num_blocks <= 0) return PKV_EINVAL;
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return PKV_EINVAL;
+  if (num_seqs == 0) return PKV_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PKV_EINVAL;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return PKV_EALIGN;
+  if (workspace && (!aligned(workspace, 16) || workspace_bytes < plan.bytes)) {
+    return aligned(workspace, 16) ? PKV_EWORKSPACE : PKV_EALIGN;
+  }
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  bool owned = false;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (!ws) {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), plan.bytes, st) != cudaSuccess) return PKV_ECUDA;
+    owned = true;
+  }
+
+  pkv::DecodeParams prm;
+  prm.q = q;
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.num_heads = num_heads;
+  prm.block_size = block_size;
+  prm.max_blocks = max_blocks_per_seq;
+  prm.num_blocks = num_blocks;
+  prm.scale_log2 = scale * pkv::kLog2e;
+  prm.part_tokens = plan.part_tokens;
+  prm.max_parts = plan.max_parts;
+  prm.out = out;
+  prm.ws_acc = plan.split ? reinterpret_cast<float*>(ws + plan.off_acc) : nullptr;
+  prm.ws_ml = plan.split ? reinterpret_cast<float2*>(ws + plan.off_ml) : nullptr;
+  prm.units = reinterpret_cast<const uint32_t*>(ws + plan.off_units);
+  prm.counters = reinterpret_cast<int*>(ws);
+
+  const int max_ctx = max_blocks_per_seq * block_size;
+  int result = PKV_OK;
+  pkv::paged_decode_plan_kernel<<<1, pkv::kPlanThreads, 0, st>>>(
+      context_lens, num_seqs, max_ctx, plan.part_tokens, reinterpret_cast<uint32_t*>(ws + plan.off_units),
+      prm.counters);
+  if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
+  const long long max_units = (long long)num_seqs * num_heads * plan.max_parts;
+  if (result == PKV_OK) {
+    result = head_dim == 64 ? dispatch_decode<64>(dtype, prm, max_units, st)
+                            : dispatch_decode<128>(dtype, prm, max_units, st);
+  }
+  if (result == PKV_OK && plan.split) {
+    const dim3 grid(num_heads, num_seqs);
+    if (head_dim == 64)
+      pkv::paged_decode_merge_kernel<64><<<grid, 128, 0, st>>>(context_lens, num_heads, max_ctx, plan.part_tokens,
+                                                               plan.max_parts, prm.ws_acc, prm.ws_ml, out);
+    else
+      pkv::paged_decode_merge_kernel<128><<<grid, 128, 0, st>>>(context_lens, num_heads, max_ctx, plan.part_tokens,
+                                                                plan.max_parts, prm.ws_acc, prm.ws_ml, out);
+    if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
+  }
+  if (owned && cudaFreeAsync(ws, st) != cudaSuccess && result == PKV_OK) result = PKV_ECUDA;
+  return result;
+}
+
+int kv_cache_append(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
+                    int num_tokens, int num_heads, int head_dim, int block_size, int num_blocks, pkv_dtype dtype,
+                    void* stream) {
+  const int e = elem_bytes(dtype);
+  if (e == 0) return PKV_EDTYPE;
+  if (num_tokens < 0 || num_heads <= 0 || num_blocks <= 0) return PKV_EINVAL;
+  if (!head_dim_ok(head_dim) || !block_size_ok(block_size)) return PKV_EUNSUPPORTED;
+  if (num_tokens == 0) return PKV_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PKV_EINVAL;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(slot_mapping, 8))
+    return PKV_EALIGN;
+  int dev;
+  if (current_device(&dev) != PKV_OK) return PKV_ECUDA;
+  const int row_vecs = head_dim * e / 16;
+  const long long total = (long long)num_tokens * 2 * num_heads * row_vecs;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  pkv::kv_append_kernel<<<grid_for(total, 256, dev), 256, 0, st>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
+      static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_heads, row_vecs, block_size,
+      (long long)num_blocks * block_size);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+int kv_block_copy(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, int num_pairs, int num_heads,
+                  int head_dim, int block_size, int num_blocks, pkv_dtype dtype, void* stream) {
+  const int e = elem_bytes(dtype);
+  if (e == 0) return PKV_EDTYPE;
+  if (num_pairs < 0 || num_heads <= 0 || num_blocks <= 0) return PKV_EINVAL;
+  if (!head_dim_ok(head_dim) || !block_size_ok(block_size)) return PKV_EUNSUPPORTED;
+  if (num_pairs == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !src_dst_pairs) return PKV_EINVAL;
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(src_dst_pairs, 8)) return PKV_EALIGN;
+  const long long block_vecs = (long long)num_heads * block_size * head_dim * e / 16;
+  const long long per_cta = (long long)pkv::kCopyThreads * pkv::kCopyVecs;
+  const long long chunks = (block_vecs + per_cta - 1) / per_cta;
+  if (chunks > INT_MAX) return PKV_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int first = 0; first < num_pairs; first += 65535) {
+    const int n = num_pairs - first < 65535 ? num_pairs - first : 65535;
+    const dim3 grid((unsigned)chunks, (unsigned)n, 2);
+    pkv::kv_block_copy_kernel<<<grid, pkv::kCopyThreads, 0, st>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), src_dst_pairs + 2 * (size_t)first, block_vecs,
+        num_blocks);
+    if (cudaGetLastError() != cudaSuccess) return PKV_ECUDA;
+  }
+  return PKV_OK;
+}
+
+int paged_kv_gather(const void* cache, const int32_t* block_table_row, int context_len, int num_heads, int head_dim,
+                    int block_size, int num_blocks, pkv_dtype dtype, void* out, void* stream) {
+  const int e = elem_bytes(dtype);
+  if (e == 0) return PKV_EDTYPE;
+  if (context_len < 0 || num_heads <= 0 || num_blocks <= 0) return PKV_EINVAL;
+  if (!head_dim_ok(head_dim) || !block_size_ok(block_size)) return PKV_EUNSUPPORTED;
+  if (context_len == 0) return PKV_OK;
+  if (!cache || !block_table_row || !out) return PKV_EINVAL;
+  if (!aligned(cache, 16) || !aligned(out, 16) || !aligned(block_table_row, 4)) return PKV_EALIGN;
+  int dev;
+  if (current_device(&dev) != PKV_OK) return PKV_ECUDA;
+  const int row_vecs = head_dim * e / 16;
+  const long long total = (long long)num_heads * context_len * row_vecs;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  pkv::kv_gather_kernel<<<grid_for(total, 256, dev), 256, 0, st>>>(
+      static_cast<const uint4*>(cache), block_table_row, context_len, num_heads, row_vecs, block_size, num_blocks,
+      static_cast<uint4*>(out));
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+int pkv_get_device_error(void* stream, int* reason) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (reason) *reason = PKV_DEV_OK;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PKV_ECUDA;
+  int word = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&word, pkv::g_error_word, sizeof(int), 0, cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  if (cudaMemcpyToSymbolAsync(pkv::g_error_word, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return PKV_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PKV_ECUDA;
+  if (reason) *reason = word;
+  if (word == PKV_DEV_OK) return PKV_OK;
+  return word == PKV_DEV_WAIT_TIMEOUT ? PKV_ETIMEOUT : PKV_EDEVICE;
+}
+
+const char* pkv_strerror(int code) {
+  switch (code) {
+    case PKV_OK: return "success";
+    case PKV_EINVAL: return "invalid argument (null pointer, size out of range or bad partition size)";
+    case PKV_EDTYPE: return "unknown storage dtype";
+    case PKV_EALIGN: return "pointer not aligned as required (16 bytes for data, 4/8 for indices)";
+    case PKV_EUNSUPPORTED: return "head_dim or block_size not supported";
+    case PKV_ECUDA: return "CUDA runtime call or kernel launch failed";
+    case PKV_EWORKSPACE: return "workspace smaller than paged_attn_decode_workspace_size()";
+    case PKV_EDEVICE: return "a kernel flagged bad device data (block id, context length, slot or copy pair)";
+    case PKV_ETIMEOUT: return "a kernel's bounded shared-memory wait ran out";
+  }
+  return "unknown error code";
+}
+
+int pkv_abi_version(void) { return 1; }
+
+}  // extern "C"

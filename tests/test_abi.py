@@ -1,0 +1,149 @@
+"""The C-ABI library: it builds, loads without a GPU, exports every declared symbol,
+and rejects bad arguments on the host before any CUDA call (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+from paged_kv_cache_328_b200 import _lib
+from paged_kv_cache_328_b200 import build as builder
+
+HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+
+PKV_OK, PKV_EINVAL, PKV_EDTYPE, PKV_EALIGN, PKV_EUNSUPPORTED = 0, -1, -2, -3, -4
+PKV_EWORKSPACE = -6
+
+
+@pytest.fixture(scope="module")
+def lib():
+    builder.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("paged_attn_decode", "kv_cache_append", "kv_block_copy", "paged_attn_decode_workspace_size",
+              "pkv_get_device_error", "pkv_strerror", "paged_kv_gather"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_library_is_built_for_sm100a_only(lib):
+    # the build command is the contract: one gencode, sm_100a
+    assert builder.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    assert os.path.exists(builder.LIB)
+
+
+def test_strerror_and_version(lib):
+    assert _lib.abi_version() == 1
+    for code in range(-8, 1):
+        assert _lib.strerror(code) != "unknown error code"
+    assert _lib.strerror(-99) == "unknown error code"
+
+
+def test_workspace_size_layout(lib):
+    # no split: counters (16) + 4 bytes per sequence rounded to 16
+    assert _lib.workspace_size(256, 40, 128, 16, 128, 2048) == 16 + 1024
+    # split into 64 partitions of 512 tokens: + m/l and acc per partition
+    n = _lib.workspace_size(8, 40, 128, 16, 2048, 512)
+    assert n == 16 + 8 * 64 * 4 + 8 * 40 * 64 * 8 + 8 * 40 * 64 * 128 * 4
+    assert _lib.partition_tokens(8, 40, 128, 16, 2048, 512) == 512
+    # the library's own choice splits long contexts into 512-token partitions
+    assert _lib.partition_tokens(8, 40, 128, 16, 2048, 0) == 512
+    # a partition as long as the longest context means no split
+    assert _lib.partition_tokens(4, 2, 64, 16, 3, 0) == 48
+
+
+@pytest.mark.parametrize("args, code", [
+    ((4, 2, 64, 16, 3, 24), PKV_EINVAL),        # not a multiple of B
+    ((4, 2, 64, 16, 3, -16), PKV_EINVAL),
+    ((4, 2, 96, 16, 3, 0), PKV_EUNSUPPORTED),   # head_dim
+    ((4, 2, 64, 12, 3, 0), PKV_EUNSUPPORTED),   # block_size
+    ((-1, 2, 64, 16, 3, 0), PKV_EINVAL),
+    ((70000, 2, 64, 16, 3, 0), PKV_EINVAL),
+    ((4, 0, 64, 16, 3, 0), PKV_EINVAL),
+])
+def test_partition_rejections(lib, args, code):
+    assert lib.paged_attn_decode_partition_tokens(*args) == code
+    assert lib.paged_attn_decode_workspace_size(*args) == ctypes.c_size_t(-1).value
+
+
+A = 0x10000  # an aligned fake device address; rejected calls never dereference it
+
+
+def decode_args(**over):
+    a = dict(q=A, k=A, v=A, bt=A, cl=A, S=4, H=2, D=64, B=16, MB=3, NB=16, dt=0, scale=0.125, out=A,
+             pt=0, ws=A, wsb=1 << 20, stream=None)
+    a.update(over)
+    return [a[k] for k in ("q", "k", "v", "bt", "cl", "S", "H", "D", "B", "MB", "NB", "dt", "scale", "out",
+                           "pt", "ws", "wsb", "stream")]
+
+
+@pytest.mark.parametrize("over, code", [
+    (dict(q=None), PKV_EINVAL),
+    (dict(out=None), PKV_EINVAL),
+    (dict(bt=None), PKV_EINVAL),
+    (dict(q=A + 8), PKV_EALIGN),
+    (dict(k=A + 4), PKV_EALIGN),
+    (dict(out=A + 4), PKV_EALIGN),
+    (dict(cl=A + 2), PKV_EALIGN),
+    (dict(ws=A + 8), PKV_EALIGN),
+    (dict(dt=7), PKV_EDTYPE),
+    (dict(D=80), PKV_EUNSUPPORTED),
+    (dict(B=24), PKV_EUNSUPPORTED),
+    (dict(pt=8), PKV_EINVAL),
+    (dict(NB=0), PKV_EINVAL),
+    (dict(scale=float("nan")), PKV_EINVAL),
+    (dict(wsb=16), PKV_EWORKSPACE),
+])
+def test_decode_rejects_on_host(lib, over, code):
+    assert lib.paged_attn_decode(*decode_args(**over)) == code
+
+
+def test_decode_empty_batch_is_a_no_op(lib):
+    assert lib.paged_attn_decode(*decode_args(S=0)) == PKV_OK
+
+
+def test_append_and_copy_reject_on_host(lib):
+    # kv_cache_append(k, v, kc, vc, slots, T, H, D, B, NB, dt, stream)
+    assert lib.kv_cache_append(A, A, A, A, A, 0, 2, 64, 16, 4, 0, None) == PKV_OK          # nothing to do
+    assert lib.kv_cache_append(None, A, A, A, A, 1, 2, 64, 16, 4, 0, None) == PKV_EINVAL
+    assert lib.kv_cache_append(A, A, A, A, A + 4, 1, 2, 64, 16, 4, 0, None) == PKV_EALIGN
+    assert lib.kv_cache_append(A, A, A, A, A, 1, 2, 48, 16, 4, 0, None) == PKV_EUNSUPPORTED
+    assert lib.kv_cache_append(A, A, A, A, A, -1, 2, 64, 16, 4, 0, None) == PKV_EINVAL
+    assert lib.kv_cache_append(A, A, A, A, A, 1, 2, 64, 16, 4, 3, None) == PKV_EDTYPE
+    # kv_block_copy(kc, vc, pairs, n, H, D, B, NB, dt, stream)
+    assert lib.kv_block_copy(A, A, A, 0, 2, 64, 16, 4, 0, None) == PKV_OK
+    assert lib.kv_block_copy(A, A, None, 1, 2, 64, 16, 4, 0, None) == PKV_EINVAL
+    assert lib.kv_block_copy(A, A + 8, A, 1, 2, 64, 16, 4, 0, None) == PKV_EALIGN
+    assert lib.kv_block_copy(A, A, A, 1, 2, 64, 17, 4, 0, None) == PKV_EUNSUPPORTED
+    # paged_kv_gather(cache, table, ctx, H, D, B, NB, dt, out, stream)
+    assert lib.paged_kv_gather(A, A, 0, 2, 64, 16, 4, 0, A, None) == PKV_OK
+    assert lib.paged_kv_gather(A, A, -1, 2, 64, 16, 4, 0, A, None) == PKV_EINVAL
+    assert lib.paged_kv_gather(A, A, 5, 2, 64, 16, 4, 0, A + 8, None) == PKV_EALIGN
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 2, 64)
+    kc = torch.zeros(4, 2, 16, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        _lib.paged_attn_decode(q, kc, kc, torch.zeros(1, 1, dtype=torch.int32),
+                               torch.zeros(1, dtype=torch.int32), 1.0,
+                               workspace=torch.zeros(64, dtype=torch.uint8))
