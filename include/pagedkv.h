@@ -204,6 +204,40 @@ const char* pkv_strerror(int code);
 /* ABI version of this header (incremented on incompatible changes). */
 int pkv_abi_version(void);
 
+/*
+ * paged_attn_decode_noalloc - paged_attn_decode for callers that cannot allocate.
+ *
+ * The pages have no counterpart to this entry point; it exists for integration.
+ * Some callers are handed only a stream and their own input/output buffers by a
+ * host framework that owns every byte of device memory (plugin-style backends),
+ * and some run latency-critical loops where a cudaMalloc, with its implicit
+ * device synchronisation and its chance of failing mid-step, is not acceptable.
+ * Neither can provide the workspace paged_attn_decode needs.  This variant
+ * computes exactly what paged_attn_decode computes, with the same arguments minus
+ * the workspace, and takes its scratch (work list, partial softmax states) from a
+ * static device array inside the library instead.  It calls no cudaMalloc,
+ * cudaFree, cudaMallocAsync or other allocating routine.
+ *
+ *  - Size limit: the scratch array holds PKV_NOALLOC_SCRATCH_BYTES (32 MiB).  A
+ *    call whose paged_attn_decode_workspace_size() exceeds it is rejected with
+ *    PKV_EWORKSPACE before anything is launched.  Every GPU that loads the
+ *    library holds this array until the process exits.
+ *  - Set-up: the first call on a device, with that device current, looks up the
+ *    array's device address (cudaGetSymbolAddress) and caches it; make that
+ *    first call on each device before any stream capture begins.
+ *  - Sharing: every call on a device uses the same array.  The call resets what
+ *    must start at zero (the work counter) itself, and the array keeps the last
+ *    call's contents.  Calls whose kernels overlap on the GPU (other streams,
+ *    other host threads) race on the array: order them on one stream.
+ *  - Return codes and device-side checks are those of paged_attn_decode.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int paged_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, const int32_t* context_lens,
+                              int num_seqs, int num_heads, int head_dim, int block_size,
+                              int max_blocks_per_seq, int num_blocks, pkv_dtype dtype,
+                              float scale, float* out, int partition_tokens, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

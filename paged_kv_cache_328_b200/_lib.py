@@ -37,7 +37,11 @@ SIGNATURES = {
     "pkv_get_device_error": (_c_int, [_c_void_p, ctypes.POINTER(_c_int)]),
     "pkv_strerror": (ctypes.c_char_p, [_c_int]),
     "pkv_abi_version": (_c_int, []),
+    "paged_attn_decode_noalloc": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                           _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                           _c_float, _c_void_p, _c_int, _c_void_p]),
 }
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class PagedKVError(RuntimeError):
@@ -214,3 +218,38 @@ def get_device_error(device=None, stream=None):
     with torch.cuda.device(dev):
         rc = lib.pkv_get_device_error(_stream(dev, stream), ctypes.byref(reason))
     return rc, reason.value
+
+
+def paged_attn_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, out=None,
+                              partition_tokens=0, stream=None):
+    """paged_attn_decode with the library's static scratch instead of a workspace.
+
+    For callers that cannot allocate device memory (a host framework that owns all
+    of it, or a loop where an allocation's synchronisation is not acceptable): the C
+    entry point allocates nothing.  ``out`` must then be passed in by such callers;
+    when it is None this wrapper creates it with torch, as a convenience for tests.
+    Calls on one device share the scratch: order them on one stream.
+    """
+    lib = load()
+    S, H, D = q.shape
+    NB, Hc, B, Dc = k_cache.shape
+    if (Hc, Dc) != (H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("q [S,H,D] and caches [NB,H,B,D] disagree")
+    if q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise TypeError("q, k_cache and v_cache must share one storage dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("block_tables must be [S, max_blocks] and context_lens [S]")
+    _cuda(q, "q", DTYPE_CODE)
+    if out is None:
+        out = torch.empty((S, H, D), dtype=torch.float32, device=q.device)
+    if out.shape != (S, H, D) or out.dtype != torch.float32:
+        raise ValueError("out must be float32 [S, H, D]")
+    args = (_cuda(q, "q", DTYPE_CODE), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+            _cuda(block_tables, "block_tables", (torch.int32,)),
+            _cuda(context_lens, "context_lens", (torch.int32,)),
+            S, H, D, B, block_tables.shape[1], NB, DTYPE_CODE[k_cache.dtype], float(scale),
+            _cuda(out, "out", (torch.float32,)), int(partition_tokens))
+    with torch.cuda.device(q.device):
+        rc = lib.paged_attn_decode_noalloc(*args, _stream(q.device, stream))
+    _check(rc, "paged_attn_decode_noalloc")
+    return out

@@ -351,3 +351,56 @@ const char* pkv_strerror(int code) {
 int pkv_abi_version(void) { return 1; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// paged_attn_decode_noalloc: the decode with its scratch in a static device
+// array, for callers that cannot allocate device memory.
+// ---------------------------------------------------------------------------
+namespace {
+
+// The scratch every paged_attn_decode_noalloc call on a device shares.  In host
+// code this name is only a stand-in for the device array; its device address
+// comes from cudaGetSymbolAddress (below).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PKV_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (the first call on a device does it) and cached.
+int noalloc_scratch(void** ptr) {
+  int dev;
+  if (current_device(&dev) != PKV_OK) return PKV_ECUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return PKV_ECUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" int paged_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                         const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                                         int num_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                                         int num_blocks, pkv_dtype dtype, float scale, float* out,
+                                         int partition_tokens, void* stream) {
+  const size_t need = paged_attn_decode_workspace_size(num_seqs, num_heads, head_dim, block_size,
+                                                       max_blocks_per_seq, partition_tokens);
+  if (need == (size_t)-1) {
+    // the same argument error paged_attn_decode reports
+    DecodePlan plan;
+    return make_plan(num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens, &plan);
+  }
+  if (need > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_EWORKSPACE;
+  if (num_seqs == 0) return PKV_OK;
+  void* scratch = nullptr;
+  const int rc = noalloc_scratch(&scratch);
+  if (rc != PKV_OK) return rc;
+  return paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads, head_dim,
+                           block_size, max_blocks_per_seq, num_blocks, dtype, scale, out, partition_tokens, scratch,
+                           (size_t)PKV_NOALLOC_SCRATCH_BYTES, stream);
+}
