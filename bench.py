@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline time budget")
+    ap.add_argument("--num-seqs", type=int, default=None,
+                    help="profiling aid: fewer sequences of the opt13b layer (a smaller case for ncu)")
     a = ap.parse_args()
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
@@ -278,7 +280,11 @@ def run_gpu(a, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     pkv.load()
 
-    w = wl.make(a.workload, device=dev, B=a.block_size if a.workload == "opt13b" else None)
+    if a.num_seqs is not None and a.workload == "opt13b":
+        w = wl.make_opt13b(B=a.block_size, device=dev, S=a.num_seqs)
+        w.name += f"_S{a.num_seqs}"
+    else:
+        w = wl.make(a.workload, device=dev, B=a.block_size if a.workload == "opt13b" else None)
     pt = w.partition_tokens if a.partition_tokens is None else a.partition_tokens
     bt = torch.from_numpy(w.block_tables).to(dev)
     ctx = torch.from_numpy(w.context_lens).to(dev)

@@ -96,11 +96,14 @@ enum {
  *   context_lens  int32 [num_seqs], 0 <= ctx <= max_blocks_per_seq * block_size.
  *   scale         multiplies q.k before the softmax (typically 1/sqrt(head_dim)).
  *   out           float32 [num_seqs][num_heads][head_dim].
- *   partition_tokens  split-context partition size in tokens: 0 = library choice;
- *                 otherwise a positive multiple of block_size.  A context longer
- *                 than one partition is processed as independent partitions whose
- *                 partial softmax states are merged exactly (log-sum-exp); a
- *                 partition size >= max_blocks_per_seq * block_size means no split.
+ *   partition_tokens  split-context partition size in tokens: 0 = library choice
+ *                 (no split when there are >= 2368 (sequence, head) pairs and
+ *                 max_blocks_per_seq * block_size <= 4096, or when that maximum is
+ *                 <= 512; otherwise 512); else a positive multiple of block_size.
+ *                 A context longer than one partition is processed as independent
+ *                 partitions whose partial softmax states are merged exactly
+ *                 (log-sum-exp); a partition size >= max_blocks_per_seq *
+ *                 block_size means no split.
  *   workspace     device scratch of at least paged_attn_decode_workspace_size()
  *                 bytes, 16-byte aligned.  It holds the call's work list (a few
  *                 bytes per sequence) and, when the call splits, the partitions'
@@ -120,8 +123,9 @@ int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
 /*
  * Workspace bytes paged_attn_decode needs for these sizes and partition_tokens
  * (0 = the library's choice, resolved exactly as paged_attn_decode resolves it):
- * 16 + 4 * num_seqs * P rounded up to 16, plus 8 * S * H * P and 4 * S * H * P *
- * head_dim (each rounded up to 16) when the call splits into P > 1 partitions.
+ * 16 + 4 * num_seqs * P rounded up to 16, plus 8 * S * H * P and
+ * 4 * S * H * P * head_dim (each rounded up to 16) when the call splits into
+ * P > 1 partitions.
  * Returns (size_t)-1 for arguments paged_attn_decode would reject.  Pure host
  * function.
  */

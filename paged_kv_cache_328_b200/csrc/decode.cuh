@@ -2,19 +2,22 @@
 //
 // Three kernels, launched back to back on one stream:
 //
-//  1. paged_decode_plan_kernel (1 CTA): turns context_lens into a compact list of
-//     live (sequence, partition) work units and resets the unit counter.
-//  2. paged_decode_kernel (persistent, one or more CTAs per SM): every CTA takes
-//     units from the counter until none are left.  A unit is (sequence s, head h,
-//     partition p).  The CTA streams the unit's K and V rows through a ring of
-//     NS shared-memory stages:
+//  1. paged_decode_plan_kernel (one CTA): turns context_lens into a compact list
+//     of live (sequence, partition) work units, longest first when the list is
+//     short enough to sort in one CTA, and resets the unit counter.
+//  2. paged_decode_kernel (persistent, launched as a programmatic dependent of
+//     the plan so that its prologue overlaps it): every CTA takes units from the
+//     counter until none are left.  A unit is (sequence s, head h, partition p).
+//     The CTA streams the unit's K and V rows through a ring of NS shared-memory
+//     stages:
 //       producer warp  follows the block table and issues one bulk (TMA-engine)
 //                      copy per contiguous (block, head) run of rows, plus the q
 //                      row at a unit's first tile; it writes a small header per
 //                      stage (unit, valid rows, first/last flags) and announces
-//                      the stage's bytes on its "full" mbarrier.  It runs ahead
-//                      across unit boundaries, so the ring never drains between
-//                      units.
+//                      the stage's bytes on its "full" mbarrier.  It reads the
+//                      table before waiting for a free stage and fetches the next
+//                      unit's list entry while streaming the current one, so the
+//                      ring does not drain between units.
 //       4 consumer warps   each 8-lane group takes one token at a time: a lane
 //                      owns D/8 dimensions, reads its 16-byte chunks of the K row
 //                      from shared memory, and the group reduces q.k with three
@@ -25,8 +28,11 @@
 //                      warps merge their states exactly and write either the
 //                      final row (single-partition context) or the partition's
 //                      (m, l, acc) to the workspace.
-//  3. paged_decode_merge_kernel: log-sum-exp merge of the partitions of every
-//     (sequence, head) whose context spans more than one partition.
+//  3. paged_decode_merge_kernel (programmatic dependent of the decode kernel):
+//     log-sum-exp merge of the partitions of every (sequence, head) whose context
+//     spans more than one partition,
+//       M = max_p m_p,  L = sum_p l_p 2^(m_p - M),  out = sum_p acc_p 2^(m_p - M) / L,
+//     which is exact algebra.
 //
 // "Gather the non-contiguous blocks along the block table and compute
 // softmax(QK^T)V" ("PagedAttention - Efficient Memory Management for LLM Serving
@@ -100,16 +106,82 @@ __device__ __forceinline__ int parts_of(int ctx, int part_tokens) {
   return n < 1 ? 1 : n;
 }
 
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------
-// 1. plan: compact list of live (sequence, partition) units.  One CTA of 1024.
+// 1. plan (one CTA).  With `sort`, one warp orders the units by decreasing
+//    length in 256-token buckets with a stable counting sort: within a bucket
+//    the units keep sequence order (partition-major within each run of 32
+//    sequences), so sequences that share prefix blocks stay adjacent and their
+//    shared blocks are re-read from L2.  Longest-first lets the dynamically
+//    scheduled CTAs end together.
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
+constexpr int kPlanBuckets = 128;
+constexpr int kPlanBucketShift = 8;  // 256 tokens per bucket
+
+__device__ __forceinline__ int unit_bucket(int len) {
+  return min(kPlanBuckets - 1, (len + (1 << kPlanBucketShift) - 1) >> kPlanBucketShift);
+}
 
 __global__ void __launch_bounds__(kPlanThreads)
     paged_decode_plan_kernel(const int32_t* __restrict__ context_lens, int num_seqs, int max_ctx, int part_tokens,
-                             uint32_t* __restrict__ units, int* __restrict__ counters) {
-  __shared__ int warp_sums[kPlanThreads / 32];
+                             int sort, uint32_t* __restrict__ units, int* __restrict__ counters) {
+  pdl_launch_dependents();
+  __shared__ int scratch[kPlanBuckets];
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+
+  if (sort) {
+    if (warp != 0) return;
+    for (int k = lane; k < kPlanBuckets; k += 32) scratch[k] = 0;
+    __syncwarp();
+    const unsigned below = (1u << lane) - 1u;
+    // pass 0 counts the units of each bucket; pass 1 places them
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int base = 0; base < num_seqs; base += 32) {
+        const int s = base + lane;
+        int ctx = 0, n = 0;
+        if (s < num_seqs) {
+          const int raw = context_lens[s];
+          if (pass == 0 && (raw < 0 || raw > max_ctx)) flag_error(PKV_DEV_CONTEXT_LEN);
+          ctx = clamp_ctx(raw, max_ctx);
+          n = parts_of(ctx, part_tokens);
+        }
+        int maxn = n;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) maxn = max(maxn, __shfl_xor_sync(0xffffffffu, maxn, o));
+        for (int p = 0; p < maxn; ++p) {
+          const bool active = p < n;
+          const int key = active ? unit_bucket(max(0, min(part_tokens, ctx - p * part_tokens))) : -1;
+          const unsigned same = __match_any_sync(0xffffffffu, key);
+          const bool leader = (same & below) == 0;
+          if (active) {
+            if (pass == 1) units[scratch[key] + __popc(same & below)] = ((uint32_t)s << 16) | (uint32_t)p;
+          }
+          __syncwarp();
+          if (active && leader) scratch[key] += __popc(same);
+          __syncwarp();
+        }
+      }
+      if (pass == 0) {  // bucket start positions, longest bucket first
+        if (lane == 0) {
+          int run = 0;
+          for (int k = kPlanBuckets - 1; k >= 0; --k) {
+            const int c = scratch[k];
+            scratch[k] = run;
+            run += c;
+          }
+          counters[0] = 0;
+          counters[1] = run;
+        }
+        __syncwarp();
+      }
+    }
+    return;
+  }
+
   const int per = (num_seqs + kPlanThreads - 1) / kPlanThreads;
   const int s0 = min(num_seqs, tid * per);
   const int s1 = min(num_seqs, s0 + per);
@@ -120,36 +192,40 @@ __global__ void __launch_bounds__(kPlanThreads)
     mine += parts_of(clamp_ctx(raw, max_ctx), part_tokens);
   }
   // exclusive scan over the CTA
-  const int lane = tid & 31, warp = tid >> 5;
   int incl = mine;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
   }
-  if (lane == 31) warp_sums[warp] = incl;
+  if (lane == 31) scratch[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_sums[lane];
+    const int w = scratch[lane];
     int wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, wi, o);
       if (lane >= o) wi += v;
     }
-    warp_sums[lane] = wi - w;  // exclusive prefix of the warp totals
+    scratch[lane] = wi - w;  // exclusive prefix of the warp totals
     if (lane == 31) {
       counters[0] = 0;
       counters[1] = wi;
     }
   }
   __syncthreads();
-  int pos = warp_sums[warp] + incl - mine;
+  int pos = scratch[warp] + incl - mine;
   for (int s = s0; s < s1; ++s) {
     const int n = parts_of(clamp_ctx(context_lens[s], max_ctx), part_tokens);
     for (int p = 0; p < n; ++p) units[pos++] = ((uint32_t)s << 16) | (uint32_t)p;
   }
 }
+
+// Unit descriptor as the producer sees it.
+struct UnitDesc {
+  int s, h, p, t_begin, t_end, n_parts;
+};
 
 // ---------------------------------------------------------------------------
 // 2. persistent decode kernel.  grid = min(#SMs x resident CTAs, units); block = 160.
@@ -182,6 +258,9 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
     fence_mbar_init();
   }
   __syncthreads();
+  // Everything above overlaps the plan kernel; the unit list, the counters and
+  // the appended cache rows are read only after it (and what precedes it) is done.
+  pdl_wait_primary();
 
   if (warp == kConsumerWarps) {
     // ------------------------------- producer -------------------------------
@@ -194,32 +273,42 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
     const int units_per_tile = TT / unit_rows;
     const long long total_units = (long long)prm.counters[1] * H;
 
+    auto describe = [&](int u, uint32_t sp) {
+      UnitDesc d{0, 0, 0, 0, 0, 1};
+      if ((long long)u < total_units) {
+        d.s = (int)(sp >> 16);
+        d.p = (int)(sp & 0xffffu);
+        d.h = u - (u / H) * H;
+        const int ctx = clamp_ctx(prm.context_lens[d.s], max_ctx);
+        d.t_begin = d.p * PT;
+        d.t_end = min(ctx, d.t_begin + PT);
+        d.n_parts = parts_of(ctx, PT);
+      }
+      return d;
+    };
+
     int u = 0;
     if (lane == 0) u = atomicAdd(&prm.counters[0], 1);
     u = __shfl_sync(0xffffffffu, u, 0);
+    UnitDesc cur = describe(u, (long long)u < total_units ? prm.units[u / H] : 0u);
     int it = 0;  // stage iterations issued so far
     bool stop = false;
     while (!stop) {
       const bool done = (long long)u >= total_units;
-      int s = 0, h = 0, p = 0, t_begin = 0, t_end = 0, n_parts = 1;
-      if (!done) {
-        const uint32_t sp = prm.units[u / H];
-        s = (int)(sp >> 16);
-        p = (int)(sp & 0xffffu);
-        h = u - (u / H) * H;
-        const int ctx = clamp_ctx(prm.context_lens[s], max_ctx);
-        t_begin = p * PT;
-        t_end = min(ctx, t_begin + PT);
-        n_parts = parts_of(ctx, PT);
-      }
       int u_next = 0;
-      if (!done && lane == 0) u_next = atomicAdd(&prm.counters[0], 1);  // used after this unit
-      const int n_tok = max(0, t_end - t_begin);
+      if (!done && lane == 0) u_next = atomicAdd(&prm.counters[0], 1);
+      uint32_t sp_next = 0;
+      const int n_tok = max(0, cur.t_end - cur.t_begin);
       const int n_tiles = done ? 1 : max(1, (n_tok + TT - 1) / TT);
-      const int32_t* table = prm.block_tables + (size_t)s * prm.max_blocks;
+      const int32_t* table = prm.block_tables + (size_t)cur.s * prm.max_blocks;
 
       for (int i = 0; i < n_tiles; ++i, ++it) {
         const int stage = it % NS;
+        // block-table entries of this tile: read before waiting for the stage
+        const int tile_t0 = cur.t_begin + i * TT;
+        const int u_t0 = tile_t0 + lane * unit_rows;
+        const bool mine = !done && lane < units_per_tile && u_t0 < cur.t_end;
+        const int phys = mine ? __ldg(table + u_t0 / B) : -1;  // u_t0 < ctx <= max_blocks * B
         if (it >= NS) {
           int ok = 1;
           if (lane == 0) ok = mbar_wait_bounded(&empty[stage], ((it / NS) - 1) & 1, abort_flag);
@@ -233,21 +322,16 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
             break;
           }
         }
-        const int tile_t0 = t_begin + i * TT;
-        const int n_valid = done ? 0 : max(0, min(TT, t_end - tile_t0));
+        const int n_valid = done ? 0 : max(0, min(TT, cur.t_end - tile_t0));
         uint32_t bytes = 0;
         size_t src_off = 0;
-        if (lane < units_per_tile) {
-          const int u_t0 = tile_t0 + lane * unit_rows;
-          if (u_t0 < t_end) {
-            const int rows = min(unit_rows, t_end - u_t0);
-            const int phys = __ldg(table + u_t0 / B);  // u_t0 < ctx <= max_blocks * B
-            if (phys >= 0 && phys < prm.num_blocks) {
-              src_off = pool_row(phys, h, u_t0 % B, H, B, D);
-              bytes = (uint32_t)rows * Tr::kRowBytes;
-            } else {
-              flag_error(PKV_DEV_BLOCK_ID);
-            }
+        if (mine) {
+          if (phys >= 0 && phys < prm.num_blocks) {
+            const int rows = min(unit_rows, cur.t_end - u_t0);
+            src_off = pool_row(phys, cur.h, u_t0 % B, H, B, D);
+            bytes = (uint32_t)rows * Tr::kRowBytes;
+          } else {
+            flag_error(PKV_DEV_BLOCK_ID);
           }
         }
         uint32_t total = bytes;
@@ -255,8 +339,8 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
         for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
         const bool load_q = (i == 0) && n_tok > 0;
         if (lane == 0) {
-          int flags = done ? kTileEnd : ((i == 0 ? kTileFirst : 0) | (i == n_tiles - 1 ? kTileLast : 0));
-          hdr[stage] = make_int4(s, h, p | (n_parts << 16), n_valid | (flags << 16));
+          const int flags = done ? kTileEnd : ((i == 0 ? kTileFirst : 0) | (i == n_tiles - 1 ? kTileLast : 0));
+          hdr[stage] = make_int4(cur.s, cur.h, cur.p | (cur.n_parts << 16), n_valid | (flags << 16));
           mbar_arrive_expect_tx(&full[stage], 2u * total + (load_q ? (uint32_t)Tr::kRowBytes : 0u));
         }
         __syncwarp();
@@ -266,13 +350,19 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
           bulk_load(st + Tr::kTileBytes, vc + src_off, bytes, &full[stage], policy);
         }
         if (load_q && lane == 0) {
-          bulk_load(smem + Tr::kQOffset + stage * Tr::kRowBytes, qg + ((size_t)s * H + h) * D, Tr::kRowBytes,
-                    &full[stage], policy);
+          bulk_load(smem + Tr::kQOffset + stage * Tr::kRowBytes, qg + ((size_t)cur.s * H + cur.h) * D,
+                    Tr::kRowBytes, &full[stage], policy);
+        }
+        if (i == 0 && !done) {  // start fetching the next unit's list entry
+          u_next = __shfl_sync(0xffffffffu, u_next, 0);
+          if ((long long)u_next < total_units) sp_next = __ldcg(prm.units + u_next / H);
         }
       }
-      if (done) break;
-      u = __shfl_sync(0xffffffffu, u_next, 0);
+      if (done || stop) break;
+      u = u_next;
+      cur = describe(u, sp_next);
     }
+    pdl_launch_dependents();  // this CTA takes no more units: the merge grid may be scheduled
     // Never leave with copies in flight into this CTA's shared memory.
     if (lane == 0) {
       int no_abort = 0;
@@ -422,20 +512,22 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
       }
       break;
     }
+    ++units_done;
+    const int us = hd.x, uh = hd.y, up = hd.z & 0xffff, un = hd.z >> 16;
+    const size_t sh = (size_t)us * H + uh;
     const int d = threadIdx.x;  // consumer thread d finalises dimension d
+    float mx = -INFINITY, L = 0.f, o = 0.f;
     if (d < D) {
-      float mx = -INFINITY;
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, rml[2 * w]);
-      float L = 0.f, o = 0.f;
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) {
         const float sc = (mx == -INFINITY) ? 0.f : exp2f(rml[2 * w] - mx);
         L = fmaf(rml[2 * w + 1], sc, L);
         o = fmaf(racc[w * D + d], sc, o);
       }
-      const int us = hd.x, uh = hd.y, up = hd.z & 0xffff, un = hd.z >> 16;
-      const size_t sh = (size_t)us * H + uh;
+    }
+    if (d < D) {
       if (un == 1) {
         prm.out[sh * D + d] = (L > 0.f) ? o / L : 0.f;
       } else {
@@ -444,14 +536,13 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
         if (d == 0) prm.ws_ml[ws] = make_float2(mx, L);
       }
     }
-    ++units_done;
   }
 }
 
 // ---------------------------------------------------------------------------
-// 3. log-sum-exp merge of the partitions of each (sequence, head):
-//      M = max_p m_p,  L = sum_p l_p 2^(m_p - M),  out = sum_p acc_p 2^(m_p - M) / L.
-//    Contexts that fit one partition were finished by the decode kernel.
+// 3. log-sum-exp merge of the partitions of each (sequence, head), one online
+//    pass over the partitions with 8 of them in flight per thread.  Contexts
+//    that fit one partition were finished by the decode kernel.
 //    grid = (num_heads, num_seqs); block = 128, thread d owns dimension d.
 // ---------------------------------------------------------------------------
 template <int D>
@@ -461,22 +552,34 @@ __global__ void __launch_bounds__(128)
                               float* __restrict__ out) {
   const int h = blockIdx.x;
   const int s = blockIdx.y;
-  const int np = parts_of(clamp_ctx(context_lens[s], max_ctx), part_tokens);
-  if (np <= 1) return;
-  const size_t sh = (size_t)s * num_heads + h;
-  const size_t base = sh * max_parts;
+  const int np = parts_of(clamp_ctx(__ldg(context_lens + s), max_ctx), part_tokens);
+  if (np <= 1) return;  // finished by the decode kernel
+  pdl_wait_primary();   // the partitions' states are complete only after the decode kernel
   const int d = threadIdx.x;
   if (d >= D) return;
-  float mx = -INFINITY;
-  for (int p = 0; p < np; ++p) mx = fmaxf(mx, ws_ml[base + p].x);
-  float L = 0.f, o = 0.f;
-  for (int p = 0; p < np; ++p) {
-    const float2 ml = ws_ml[base + p];
-    const float sc = (mx == -INFINITY) ? 0.f : exp2f(ml.x - mx);
-    L = fmaf(ml.y, sc, L);
-    o = fmaf(ws_acc[(base + p) * D + d], sc, o);
+  const size_t base = ((size_t)s * num_heads + h) * max_parts;
+  float M = -INFINITY, L = 0.f, o = 0.f;
+  for (int p0 = 0; p0 < np; p0 += 8) {
+    float2 ml[8];
+    float a[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool in = p0 + j < np;
+      ml[j] = in ? __ldcg(ws_ml + base + p0 + j) : make_float2(-INFINITY, 0.f);
+      a[j] = in ? __ldcg(ws_acc + (base + p0 + j) * D + d) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float mn = fmaxf(M, ml[j].x);
+      if (mn == -INFINITY) continue;
+      const float keep = exp2f(M - mn);     // 0 while M is -inf
+      const float add = exp2f(ml[j].x - mn);
+      L = L * keep + ml[j].y * add;
+      o = o * keep + a[j] * add;
+      M = mn;
+    }
   }
-  out[sh * D + d] = (L > 0.f) ? o / L : 0.f;
+  out[((size_t)s * num_heads + h) * D + d] = (L > 0.f) ? o / L : 0.f;
 }
 
 }  // namespace pkv

@@ -2,8 +2,9 @@
 //
 // Host side only: argument validation (before any CUDA call), resolution of the
 // split-context partition size, workspace layout, and kernel launches.  The
-// kernels live in decode.cuh (paged decode attention: plan, persistent decode,
-// log-sum-exp merge) and cache_ops.cuh (append, block copy, gather).
+// kernels live in decode.cuh (paged decode attention: plan, persistent decode
+// with the log-sum-exp merge of split contexts) and cache_ops.cuh (append, block
+// copy, gather).
 #include <climits>
 #include <cstdint>
 #include <cstring>
@@ -41,14 +42,22 @@ struct DecodePlan {
   int part_tokens = 0;
   int max_parts = 1;
   bool split = false;
+  bool sort = false;
   size_t off_units = 0, off_ml = 0, off_acc = 0, bytes = 0;
 };
 
-// Library choice of partition size when the caller passes 0: contexts longer than
-// 512 tokens are split into 512-token partitions (a multiple of every supported
-// block size), which bounds the work of one unit so that the persistent CTAs
-// finish together; shorter maximum contexts are not split.
+// Library choice of partition size when the caller passes 0.  The persistent
+// grid holds about kRefCtas CTAs (148 SMs x 2).  When there are at least 8 (sequence,
+// head) units per CTA and no context exceeds 4096 tokens, the longest-first unit
+// order already balances the CTAs and splitting would only add partial-state
+// traffic, so contexts are not split.  Otherwise contexts are cut into 512-token
+// partitions (a multiple of every supported block size), which bounds the work
+// of one unit.  Maximum contexts of at most 512 tokens are never split.
 constexpr int kAutoPartitionTokens = 512;
+constexpr long long kRefCtas = 148 * 2;
+// Unit lists up to this length are ordered longest first by the plan kernel
+// (one warp, 32 units per step).
+constexpr long long kSortedUnitsMax = 4096;
 
 int make_plan(int S, int H, int D, int B, int MB, int requested, DecodePlan* plan) {
   if (S < 0 || H <= 0 || MB <= 0) return PKV_EINVAL;
@@ -57,7 +66,11 @@ int make_plan(int S, int H, int D, int B, int MB, int requested, DecodePlan* pla
   const long long max_ctx = (long long)MB * B;
   if (max_ctx > (INT_MAX / 2)) return PKV_EINVAL;
   if (requested < 0 || (requested > 0 && requested % B != 0)) return PKV_EINVAL;
-  long long pt = requested > 0 ? requested : kAutoPartitionTokens;
+  long long pt = requested;
+  if (requested == 0) {
+    const bool enough_units = (long long)S * H >= 8 * kRefCtas && max_ctx <= 4096;
+    pt = (max_ctx <= kAutoPartitionTokens || enough_units) ? max_ctx : kAutoPartitionTokens;
+  }
   if (pt >= max_ctx) pt = max_ctx;
   const long long parts = (max_ctx + pt - 1) / pt;
   if (parts > 32767) return PKV_EINVAL;
@@ -65,6 +78,7 @@ int make_plan(int S, int H, int D, int B, int MB, int requested, DecodePlan* pla
   plan->part_tokens = (int)pt;
   plan->max_parts = (int)parts;
   plan->split = parts > 1;
+  plan->sort = (long long)S * parts <= kSortedUnitsMax;
   size_t off = 16;  // counters[2] (+ padding)
   plan->off_units = off;
   off += round16((size_t)S * parts * sizeof(uint32_t));
@@ -130,7 +144,19 @@ int launch_decode(const pkv::DecodeParams& prm, long long max_units, cudaStream_
   long long grid = (long long)sms * occ;
   if (grid > max_units) grid = max_units;
   if (grid < 1) grid = 1;
-  pkv::paged_decode_kernel<T, D, TT, NS><<<(unsigned)grid, pkv::kDecodeThreads, Tr::kSmemBytes, st>>>(prm);
+  // Programmatic dependent launch: the CTAs start while the plan kernel runs and
+  // wait for it (griddepcontrol.wait) after their prologue.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(pkv::kDecodeThreads);
+  cfg.dynamicSmemBytes = Tr::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, pkv::paged_decode_kernel<T, D, TT, NS>, prm) != cudaSuccess) return PKV_ECUDA;
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
 
@@ -146,6 +172,27 @@ int dispatch_decode(pkv_dtype dt, const pkv::DecodeParams& prm, long long max_un
     case PKV_F32: return launch_decode<float, D, kTT32, 3>(prm, max_units, st);
   }
   return PKV_EDTYPE;
+}
+
+// The merge is a programmatic dependent of the decode kernel: its CTAs may be
+// scheduled as decode CTAs run out of units and wait for the decode to finish.
+template <int D>
+int launch_merge(const int32_t* context_lens, int S, int H, int max_ctx, const DecodePlan& plan, const float* ws_acc,
+                 const float2* ws_ml, float* out, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)H, (unsigned)S);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, pkv::paged_decode_merge_kernel<D>, context_lens, H, max_ctx, plan.part_tokens,
+                         plan.max_parts, ws_acc, ws_ml, out) != cudaSuccess)
+    return PKV_ECUDA;
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
 
 int grid_for(long long work, int per_block, int dev) {
@@ -225,8 +272,8 @@ int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache, c
   const int max_ctx = max_blocks_per_seq * block_size;
   int result = PKV_OK;
   pkv::paged_decode_plan_kernel<<<1, pkv::kPlanThreads, 0, st>>>(
-      context_lens, num_seqs, max_ctx, plan.part_tokens, reinterpret_cast<uint32_t*>(ws + plan.off_units),
-      prm.counters);
+      context_lens, num_seqs, max_ctx, plan.part_tokens, plan.sort ? 1 : 0,
+      reinterpret_cast<uint32_t*>(ws + plan.off_units), prm.counters);
   if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
   const long long max_units = (long long)num_seqs * num_heads * plan.max_parts;
   if (result == PKV_OK) {
@@ -234,14 +281,9 @@ int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache, c
                             : dispatch_decode<128>(dtype, prm, max_units, st);
   }
   if (result == PKV_OK && plan.split) {
-    const dim3 grid(num_heads, num_seqs);
-    if (head_dim == 64)
-      pkv::paged_decode_merge_kernel<64><<<grid, 128, 0, st>>>(context_lens, num_heads, max_ctx, plan.part_tokens,
-                                                               plan.max_parts, prm.ws_acc, prm.ws_ml, out);
-    else
-      pkv::paged_decode_merge_kernel<128><<<grid, 128, 0, st>>>(context_lens, num_heads, max_ctx, plan.part_tokens,
-                                                                plan.max_parts, prm.ws_acc, prm.ws_ml, out);
-    if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
+    result = head_dim == 64
+                 ? launch_merge<64>(context_lens, num_seqs, num_heads, max_ctx, plan, prm.ws_acc, prm.ws_ml, out, st)
+                 : launch_merge<128>(context_lens, num_seqs, num_heads, max_ctx, plan, prm.ws_acc, prm.ws_ml, out, st);
   }
   if (owned && cudaFreeAsync(ws, st) != cudaSuccess && result == PKV_OK) result = PKV_ECUDA;
   return result;
