@@ -7,37 +7,31 @@
 
 namespace pkv {
 
-// kv_cache_append: one thread per 16-byte vector of one (token, K|V, head) row.
-// row_vecs = head_dim * elem_bytes / 16.  Grid-stride over
-// num_tokens * 2 * num_heads * row_vecs vectors.
-__global__ void __launch_bounds__(256)
+// kv_cache_append: grid = (num_tokens, 2 for K|V); the CTA of token t copies its
+// num_heads rows of row_vecs 16-byte vectors into the slot's rows (one per head).
+constexpr int kAppendThreads = 128;
+
+__global__ void __launch_bounds__(kAppendThreads)
     kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, uint4* __restrict__ k_cache,
-                     uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int num_tokens,
-                     int num_heads, int row_vecs, int block_size, long long num_slots) {
-  const long long per_token = 2LL * num_heads * row_vecs;
-  const long long total = (long long)num_tokens * per_token;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int t = (int)(i / per_token);
-    long long r = i - (long long)t * per_token;
-    const int is_v = (int)(r / ((long long)num_heads * row_vecs));
-    r -= (long long)is_v * num_heads * row_vecs;
-    const int h = (int)(r / row_vecs);
-    const int vec = (int)(r - (long long)h * row_vecs);
-    const long long slot = slot_mapping[t];
-    if (slot < 0) continue;
-    if (slot >= num_slots) {
-      if (is_v == 0 && h == 0 && vec == 0) flag_error(PKV_DEV_SLOT);
-      continue;
-    }
-    const long long blk = slot / block_size;
-    const long long off = slot - blk * block_size;
-    const size_t dst = pool_row(blk, h, off, num_heads, block_size, row_vecs) + vec;
-    const size_t src = ((size_t)t * num_heads + h) * row_vecs + vec;
-    if (is_v)
-      v_cache[dst] = v_new[src];
-    else
-      k_cache[dst] = k_new[src];
+                     uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int num_heads,
+                     int row_vecs, int block_size, long long num_slots) {
+  const int t = blockIdx.x;
+  const int is_v = blockIdx.y;
+  const long long slot = slot_mapping[t];
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (is_v == 0 && threadIdx.x == 0) flag_error(PKV_DEV_SLOT);
+    return;
+  }
+  const long long blk = slot / block_size;
+  const int off = (int)(slot - blk * block_size);
+  const int per_token = num_heads * row_vecs;
+  const uint4* src = (is_v ? v_new : k_new) + (size_t)t * per_token;
+  uint4* cache = is_v ? v_cache : k_cache;
+  for (int i = threadIdx.x; i < per_token; i += kAppendThreads) {
+    const int h = i / row_vecs;
+    const int vec = i - h * row_vecs;
+    cache[pool_row(blk, h, off, num_heads, block_size, row_vecs) + vec] = src[i];
   }
 }
 

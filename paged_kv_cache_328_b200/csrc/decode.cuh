@@ -112,14 +112,14 @@ __device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontro
 // ---------------------------------------------------------------------------
 // 1. plan (one CTA).  With `sort`, one warp orders the units by decreasing
 //    length in 256-token buckets with a stable counting sort: within a bucket
-//    the units keep sequence order (partition-major within each run of 32
-//    sequences), so sequences that share prefix blocks stay adjacent and their
-//    shared blocks are re-read from L2.  Longest-first lets the dynamically
-//    scheduled CTAs end together.
+//    the units keep sequence order, so sequences that share prefix blocks stay
+//    adjacent and their shared blocks are re-read from L2.  Longest-first lets
+//    the dynamically scheduled CTAs end together.
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 128;
 constexpr int kPlanBucketShift = 8;  // 256 tokens per bucket
+constexpr int kPlanSortMaxSeqs = 4096;  // sorted lists: num_seqs * partitions <= this
 
 __device__ __forceinline__ int unit_bucket(int len) {
   return min(kPlanBuckets - 1, (len + (1 << kPlanBucketShift) - 1) >> kPlanBucketShift);
@@ -134,36 +134,48 @@ __global__ void __launch_bounds__(kPlanThreads)
   const int lane = tid & 31, warp = tid >> 5;
 
   if (sort) {
+    // the lengths go through shared memory once (num_seqs <= kPlanSortMaxSeqs)
+    __shared__ int ctx_s[kPlanSortMaxSeqs];
+    for (int s = tid; s < num_seqs; s += kPlanThreads) {
+      const int raw = context_lens[s];
+      if (raw < 0 || raw > max_ctx) flag_error(PKV_DEV_CONTEXT_LEN);
+      ctx_s[s] = clamp_ctx(raw, max_ctx);
+    }
+    for (int k = tid; k < kPlanBuckets; k += kPlanThreads) scratch[k] = 0;
+    __syncthreads();
     if (warp != 0) return;
-    for (int k = lane; k < kPlanBuckets; k += 32) scratch[k] = 0;
-    __syncwarp();
     const unsigned below = (1u << lane) - 1u;
-    // pass 0 counts the units of each bucket; pass 1 places them
+    const int key_full = unit_bucket(part_tokens);  // every partition but a sequence's last is full
+    // pass 0 counts the units of each bucket; pass 1 places them.  A run of 32
+    // sequences places its full partitions (sequence-major) then its last ones.
     for (int pass = 0; pass < 2; ++pass) {
       for (int base = 0; base < num_seqs; base += 32) {
         const int s = base + lane;
-        int ctx = 0, n = 0;
-        if (s < num_seqs) {
-          const int raw = context_lens[s];
-          if (pass == 0 && (raw < 0 || raw > max_ctx)) flag_error(PKV_DEV_CONTEXT_LEN);
-          ctx = clamp_ctx(raw, max_ctx);
-          n = parts_of(ctx, part_tokens);
-        }
-        int maxn = n;
+        const bool live = s < num_seqs;
+        const int ctx = live ? ctx_s[s] : 0;
+        const int n = live ? parts_of(ctx, part_tokens) : 0;
+        const int nfull = max(n - 1, 0);
+        int excl = nfull;  // exclusive scan of nfull over the warp
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) maxn = max(maxn, __shfl_xor_sync(0xffffffffu, maxn, o));
-        for (int p = 0; p < maxn; ++p) {
-          const bool active = p < n;
-          const int key = active ? unit_bucket(max(0, min(part_tokens, ctx - p * part_tokens))) : -1;
-          const unsigned same = __match_any_sync(0xffffffffu, key);
-          const bool leader = (same & below) == 0;
-          if (active) {
-            if (pass == 1) units[scratch[key] + __popc(same & below)] = ((uint32_t)s << 16) | (uint32_t)p;
-          }
-          __syncwarp();
-          if (active && leader) scratch[key] += __popc(same);
-          __syncwarp();
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, excl, o);
+          if (lane >= o) excl += v;
         }
+        const int tot = __shfl_sync(0xffffffffu, excl, 31);
+        excl -= nfull;
+        if (pass == 1) {
+          const int at = scratch[key_full] + excl;
+          for (int j = 0; j < nfull; ++j) units[at + j] = ((uint32_t)s << 16) | (uint32_t)j;
+        }
+        __syncwarp();
+        if (lane == 0 && tot > 0) scratch[key_full] += tot;
+        __syncwarp();
+        const int key = live ? unit_bucket(ctx - (n - 1) * part_tokens) : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, key);
+        if (live && pass == 1) units[scratch[key] + __popc(same & below)] = ((uint32_t)s << 16) | (uint32_t)(n - 1);
+        __syncwarp();
+        if (live && (same & below) == 0) scratch[key] += __popc(same);
+        __syncwarp();
       }
       if (pass == 0) {  // bucket start positions, longest bucket first
         if (lane == 0) {

@@ -56,8 +56,8 @@ struct DecodePlan {
 constexpr int kAutoPartitionTokens = 512;
 constexpr long long kRefCtas = 148 * 2;
 // Unit lists up to this length are ordered longest first by the plan kernel
-// (one warp, 32 units per step).
-constexpr long long kSortedUnitsMax = 4096;
+// (one warp, 32 sequences per step; the lengths are staged in shared memory).
+constexpr long long kSortedUnitsMax = pkv::kPlanSortMaxSeqs;
 
 int make_plan(int S, int H, int D, int B, int MB, int requested, DecodePlan* plan) {
   if (S < 0 || H <= 0 || MB <= 0) return PKV_EINVAL;
@@ -303,12 +303,13 @@ int kv_cache_append(const void* k, const void* v, void* k_cache, void* v_cache, 
     return PKV_EALIGN;
   int dev;
   if (current_device(&dev) != PKV_OK) return PKV_ECUDA;
+  (void)dev;
   const int row_vecs = head_dim * e / 16;
-  const long long total = (long long)num_tokens * 2 * num_heads * row_vecs;
+  if ((long long)num_heads * row_vecs > INT_MAX) return PKV_EINVAL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  pkv::kv_append_kernel<<<grid_for(total, 256, dev), 256, 0, st>>>(
+  pkv::kv_append_kernel<<<dim3((unsigned)num_tokens, 2), pkv::kAppendThreads, 0, st>>>(
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
-      static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_heads, row_vecs, block_size,
+      static_cast<uint4*>(v_cache), slot_mapping, num_heads, row_vecs, block_size,
       (long long)num_blocks * block_size);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
