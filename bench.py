@@ -246,7 +246,8 @@ class ClockSampler:
 # The GPU arm
 # ---------------------------------------------------------------------------
 def traffic_record(workload_key):
-    """dram bytes per decode launch from a committed ncu capture, if the kernel sources are unchanged."""
+    """dram bytes per decode launch from a committed ncu capture, if the decode kernel's sources
+    (listed in the record) are unchanged since the capture; else None."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
@@ -256,8 +257,8 @@ def traffic_record(workload_key):
     if not rec:
         return None
     h = hashlib.sha256()
-    for f in sorted(os.listdir(os.path.join(ROOT, "paged_kv_cache_328_b200", "csrc"))):
-        h.update(open(os.path.join(ROOT, "paged_kv_cache_328_b200", "csrc", f), "rb").read())
+    for f in rec.get("kernel_sources", []):
+        h.update(open(os.path.join(ROOT, f), "rb").read())
     return rec["dram_bytes_per_launch"] if rec.get("csrc_sha256") == h.hexdigest() else None
 
 

@@ -97,7 +97,7 @@ enum {
  *   scale         multiplies q.k before the softmax (typically 1/sqrt(head_dim)).
  *   out           float32 [num_seqs][num_heads][head_dim].
  *   partition_tokens  split-context partition size in tokens: 0 = library choice
- *                 (no split when there are >= 2368 (sequence, head) pairs and
+ *                 (no split when there are >= 1184 (sequence, head) pairs and
  *                 max_blocks_per_seq * block_size <= 4096, or when that maximum is
  *                 <= 512; otherwise 512); else a positive multiple of block_size.
  *                 A context longer than one partition is processed as independent

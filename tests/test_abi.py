@@ -70,7 +70,8 @@ def test_workspace_size_layout(lib):
     assert _lib.partition_tokens(4, 2, 64, 16, 3, 0) == 48
     # enough (sequence, head) pairs and contexts <= 4096: no split by default
     assert _lib.partition_tokens(256, 40, 128, 16, 128, 0) == 2048
-    assert _lib.partition_tokens(64, 32, 128, 16, 128, 0) == 512      # 2048 pairs: split
+    assert _lib.partition_tokens(64, 32, 128, 16, 128, 0) == 2048     # 2048 pairs: no split
+    assert _lib.partition_tokens(32, 32, 128, 16, 128, 0) == 512      # 1024 pairs: split
     assert _lib.partition_tokens(256, 40, 128, 16, 512, 0) == 512     # contexts up to 8192: split
 
 
