@@ -24,6 +24,10 @@ Readings where the pages are silent:
 * The scale multiplies q.k before the softmax (1/sqrt(head_dim) in the workloads).
 * A context of length 0 gives an all-zero output.
 * Slots at or beyond the context length, and blocks not in the table, are never read.
+* Grouped-query attention (fewer K/V heads than query heads, named on the digest's
+  related-work list as an orthogonal way to shrink the KV cache): with Hq query
+  heads and Hkv K/V heads, G = Hq / Hkv consecutive query heads share one K/V head,
+  query head h reading K/V head h // G.  Hkv = Hq is ordinary multi-head attention.
 """
 
 import numpy as np
@@ -81,23 +85,29 @@ def attend(q, K, V, scale):
 
 def paged_decode_selected(q, k_pool, v_pool, block_tables, context_lens, scale,
                           block_size, dtype, selection):
-    """Decode outputs for the listed (sequence, head) pairs only: float64 ``[len(selection), D]``.
+    """Decode outputs for the listed (sequence, query head) pairs: float64 ``[len(selection), D]``.
 
-    ``q`` is ``[S, H, D]`` and the pools ``[NB, H, B, D]``, all stored in ``dtype``.
+    ``q`` is ``[S, Hq, D]`` and the pools ``[NB, Hkv, B, D]``, all stored in ``dtype``;
+    Hq must be a multiple of Hkv and query head h reads K/V head h // (Hq // Hkv).
     """
-    D = q.shape[2]
+    Hq, D = q.shape[1], q.shape[2]
+    Hkv = k_pool.shape[1]
+    if Hq % Hkv:
+        raise ValueError("query heads must be a multiple of K/V heads")
+    group = Hq // Hkv
     out = np.zeros((len(selection), D), dtype=np.float64)
     for i, (s, h) in enumerate(selection):
         ctx = int(context_lens[s])
-        K = to_f64(gather_rows(k_pool, block_tables[s], ctx, h, block_size), dtype)
-        V = to_f64(gather_rows(v_pool, block_tables[s], ctx, h, block_size), dtype)
+        kvh = h // group
+        K = to_f64(gather_rows(k_pool, block_tables[s], ctx, kvh, block_size), dtype)
+        V = to_f64(gather_rows(v_pool, block_tables[s], ctx, kvh, block_size), dtype)
         qv = to_f64(q[s, h], dtype)
         out[i] = attend(qv, K, V, scale)
     return out
 
 
 def paged_decode(q, k_pool, v_pool, block_tables, context_lens, scale, block_size, dtype):
-    """Decode outputs for every sequence and head: float64 ``[S, H, D]``."""
+    """Decode outputs for every sequence and query head: float64 ``[S, Hq, D]``."""
     S, H, D = q.shape
     sel = [(s, h) for s in range(S) for h in range(H)]
     flat = paged_decode_selected(q, k_pool, v_pool, block_tables, context_lens, scale,

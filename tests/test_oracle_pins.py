@@ -440,6 +440,29 @@ def check_block_copy_brute_force():
     assert np.array_equal(k2.reshape(-1), kf) and np.array_equal(v2.reshape(-1), vf)
 
 
+def check_gqa_equals_replicated_mha():
+    """Grouped-query attention is multi-head attention with each K/V head repeated G times."""
+    rng = np.random.default_rng(22)
+    Hq, Hkv, D, B, nb, ctx = 8, 2, 64, 16, 12, 70
+    G = Hq // Hkv
+    for dtype in ("f16", "bf16"):
+        K = random_stored(rng, (Hkv, ctx, D), dtype)
+        V = random_stored(rng, (Hkv, ctx, D), dtype)
+        q = random_stored(rng, (1, Hq, D), dtype)
+        table = random_table(rng, nb, -(-ctx // B))
+        kp, vp = place_flat(K, V, B, nb, table, dtype)
+        kr, vr = place_flat(np.repeat(K, G, axis=0), np.repeat(V, G, axis=0), B, nb, table, dtype)
+        gqa = oracle.paged_decode(q, kp, vp, np.array([table]), np.array([ctx]), 0.125, B, dtype)
+        mha = oracle.paged_decode(q, kr, vr, np.array([table]), np.array([ctx]), 0.125, B, dtype)
+        assert np.array_equal(gqa, mha)
+        # and against the library routine, grouped the same way
+        qt = torch.from_numpy(storage_lib(q[0], dtype))[:, None, :]
+        Kt = torch.from_numpy(storage_lib(K, dtype)).repeat_interleave(G, dim=0)
+        Vt = torch.from_numpy(storage_lib(V, dtype)).repeat_interleave(G, dim=0)
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, scale=0.125)[:, 0, :]
+        assert np.max(np.abs(gqa[0] - ref.numpy())) <= 1e-12
+
+
 def all_pin_checks(golden_dir):
     return [
         check_storage_f16,
@@ -460,6 +483,7 @@ def all_pin_checks(golden_dir):
         check_block_size_invariance,
         check_append_brute_force,
         check_block_copy_brute_force,
+        check_gqa_equals_replicated_mha,
     ]
 
 
@@ -532,6 +556,10 @@ def test_block_copy_brute_force():
     check_block_copy_brute_force()
 
 
+def test_gqa_equals_replicated_mha():
+    check_gqa_equals_replicated_mha()
+
+
 def test_softmax_weights_sum_to_one():
     rng = np.random.default_rng(21)
     for n in (1, 2, 7, 1000):
@@ -561,6 +589,19 @@ def _mut_div_mod_swapped(pool, table_row, ctx, head, block_size):
 
 def _mut_mask_short(pool, table_row, ctx, head, block_size):
     return _orig_gather_rows(pool, table_row, max(int(ctx) - 1, 0) if ctx > 1 else ctx, head, block_size)
+
+
+def _mut_gqa_head_modulo(q, k_pool, v_pool, block_tables, context_lens, scale, block_size, dtype, selection):
+    """Reads K/V head h % Hkv instead of h // G (a plausible grouping mistake)."""
+    Hkv = k_pool.shape[1]
+    D = q.shape[2]
+    out = np.zeros((len(selection), D))
+    for i, (s, h) in enumerate(selection):
+        ctx = int(context_lens[s])
+        K = storage.to_f64(_orig_gather_rows(k_pool, block_tables[s], ctx, h % Hkv, block_size), dtype)
+        V = storage.to_f64(_orig_gather_rows(v_pool, block_tables[s], ctx, h % Hkv, block_size), dtype)
+        out[i] = _orig_attend(storage.to_f64(q[s, h], dtype), K, V, scale)
+    return out
 
 
 def _mut_no_scale(q, K, V, scale):
@@ -602,6 +643,7 @@ MUTANTS = {
     "bf16 decoded as fp16": [(storage, "to_f64", "bf16_as_f16")],
     "append block/offset swapped": [(cache_ops, "kv_append", _mut_append_div_mod_swapped)],
     "block copy forgets V": [(cache_ops, "kv_block_copy", _mut_copy_k_only)],
+    "query head grouped by modulo": [(paged_attention, "paged_decode_selected", _mut_gqa_head_modulo)],
 }
 
 
