@@ -37,8 +37,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention effective KV GB/s and % of B200 HBM peak"
 FALLBACK_HBM_GBS = 6650.0
-WORKLOADS = ("opt13b", "llama7b", "cow", "longctx", "tiny")
-DEFAULT_STEPS = {"opt13b": 500, "llama7b": 2000, "cow": 1000, "longctx": 500, "tiny": 200}
+WORKLOADS = ("opt13b", "llama7b", "cow", "longctx", "tiny", "gqa2", "gqa4", "gqa8", "gqa16")
+DEFAULT_STEPS = {"opt13b": 500, "llama7b": 2000, "cow": 1000, "longctx": 500, "tiny": 200,
+                 "gqa2": 500, "gqa4": 500, "gqa8": 500, "gqa16": 500}
 
 
 def parse():
@@ -127,11 +128,16 @@ def make_cpu_sample(wname, block_size, n_seq, seed=7):
               "cow": (40, 128, "f16", None), "longctx": (40, 128, "f16", wl.uniform_lengths(8, wl.BASE_SEED + 5,
                                                                                          16384, 32768)),
               "tiny": (2, 64, "f32", wl.tiny_lengths())}
+    Hq = None
+    if wname.startswith("gqa"):  # 8 K/V heads shared by `group` query heads each
+        shapes[wname] = (8, 128, "bf16", wl.opt13b_lengths())
+        Hq = 8 * int(wname[3:])
     H, D, dtype, ctx = shapes[wname]
+    Hq = H if Hq is None else Hq
     if ctx is None:
         rng = np.random.default_rng(wl.BASE_SEED + 4)
         ctx = 512 + rng.integers(1, 257, size=128) + 1
-    B = block_size if wname == "opt13b" else (16 if wname != "tiny" else 16)
+    B = block_size if (wname == "opt13b" or wname.startswith("gqa")) else 16
     rng = np.random.default_rng(seed)
     cases = []
     for c in [int(x) for x in ctx[:n_seq]]:
@@ -141,11 +147,11 @@ def make_cpu_sample(wname, block_size, n_seq, seed=7):
         if dtype == "f32":
             k = rng.standard_normal((nb, H, B, D), dtype=np.float32)
             v = rng.standard_normal((nb, H, B, D), dtype=np.float32)
-            q = rng.standard_normal((1, H, D), dtype=np.float32)
+            q = rng.standard_normal((1, Hq, D), dtype=np.float32)
         else:
             k = rng.integers(0, 1 << 16, size=(nb, H, B, D), dtype=np.uint16) & np.uint16(0xBFFF)
             v = rng.integers(0, 1 << 16, size=(nb, H, B, D), dtype=np.uint16) & np.uint16(0xBFFF)
-            q = rng.integers(0, 1 << 16, size=(1, H, D), dtype=np.uint16) & np.uint16(0xBFFF)
+            q = rng.integers(0, 1 << 16, size=(1, Hq, D), dtype=np.uint16) & np.uint16(0xBFFF)
             if dtype == "f16":  # keep magnitudes moderate: exponent field <= 15
                 k, v, q = (x & np.uint16(0xBBFF) for x in (k, v, q))
         cases.append(dict(q=q, k=k, v=v, table=table, ctx=np.array([c]), nbytes=c * H * D * (2 if dtype != "f32"
@@ -285,7 +291,8 @@ def run_gpu(a, rank, world, local_rank):
         w = wl.make_opt13b(B=a.block_size, device=dev, S=a.num_seqs)
         w.name += f"_S{a.num_seqs}"
     else:
-        w = wl.make(a.workload, device=dev, B=a.block_size if a.workload == "opt13b" else None)
+        w = wl.make(a.workload, device=dev, B=a.block_size if a.workload in ("opt13b",) or
+                    a.workload.startswith("gqa") else None)
     pt = w.partition_tokens if a.partition_tokens is None else a.partition_tokens
     bt = torch.from_numpy(w.block_tables).to(dev)
     ctx = torch.from_numpy(w.context_lens).to(dev)
@@ -293,7 +300,8 @@ def run_gpu(a, rank, world, local_rank):
     pairs = torch.from_numpy(w.cow_pairs.reshape(-1, 2)).to(dev)
     out = torch.empty((w.S, w.H, w.D), dtype=torch.float32, device=dev)
     ws = pkv.alloc_workspace(w.q, w.k_pool, bt, pt)
-    split = pkv.partition_tokens(w.S, w.H, w.D, w.B, w.max_blocks, pt) < w.max_blocks * w.B
+    pt_used = pkv.gqa_partition_tokens(w.S, w.H, w.Hkv, w.D, w.B, w.max_blocks, pt)
+    split = pt_used < w.max_blocks * w.B
     stream = torch.cuda.current_stream(dev)
     launches_per_step = (1 if len(w.cow_pairs) else 0) + 1 + 2 + (1 if split else 0)
 
@@ -403,10 +411,11 @@ def run_gpu(a, rank, world, local_rank):
         "dtype": w.dtype,
         "data": "synthetic",
         "config": {
-            "workload": w.name, "num_seqs": w.S, "num_heads": w.H, "head_dim": w.D, "block_size": w.B,
+            "workload": w.name, "num_seqs": w.S, "num_heads": w.H, "num_kv_heads": w.Hkv, "head_dim": w.D,
+            "block_size": w.B,
             "context_tokens_per_step": int(w.context_lens.sum()), "kv_bytes_per_step": kv_bytes,
             "cow_pairs_per_step": int(len(w.cow_pairs)), "appended_tokens_per_step": int((w.slot_mapping >= 0).sum()),
-            "partition_tokens": pkv.partition_tokens(w.S, w.H, w.D, w.B, w.max_blocks, pt),
+            "partition_tokens": pt_used,
             "l2": f"no flush: K/V pool {w.k_pool.numel() * w.k_pool.element_size() * 2 / 1e9:.2f} GB "
                   f"= {w.k_pool.numel() * w.k_pool.element_size() * 2 / 126e6:.0f}x L2",
             "parallelism": f"replicas x{world}",

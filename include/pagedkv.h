@@ -142,6 +142,40 @@ int paged_attn_decode_partition_tokens(int num_seqs, int num_heads, int head_dim
                                        int partition_tokens);
 
 /*
+ * paged_attn_decode_gqa - paged_attn_decode for grouped-query attention.
+ *
+ * num_heads query heads share num_kv_heads K/V heads (num_heads a multiple of
+ * num_kv_heads): query head h reads K/V head h / (num_heads / num_kv_heads).  The
+ * digest ("PagedAttention - Efficient Memory Management for LLM Serving with
+ * vLLM", related work) names fewer K/V heads (GQA) as a way to shrink the KV cache
+ * that is orthogonal to paging.
+ *
+ *   q, out        [num_seqs][num_heads][head_dim] (q in the storage dtype, out fp32).
+ *   k_cache,
+ *   v_cache       [num_blocks][num_kv_heads][block_size][head_dim].
+ *   Every other argument, the return codes and the device-side checks are those of
+ *   paged_attn_decode; num_kv_heads == num_heads is exactly paged_attn_decode.
+ *   The workspace size comes from paged_attn_decode_gqa_workspace_size.
+ */
+int paged_attn_decode_gqa(const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens,
+                          int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                          int block_size, int max_blocks_per_seq, int num_blocks,
+                          pkv_dtype dtype, float scale, float* out, int partition_tokens,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes paged_attn_decode_gqa needs; (size_t)-1 for rejected arguments. */
+size_t paged_attn_decode_gqa_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                            int head_dim, int block_size,
+                                            int max_blocks_per_seq, int partition_tokens);
+
+/* Partition size paged_attn_decode_gqa will use (the library's choice counts
+ * (sequence, K/V head) pairs), or a negative PKV_E* code.  Pure host function. */
+int paged_attn_decode_gqa_partition_tokens(int num_seqs, int num_heads, int num_kv_heads,
+                                           int head_dim, int block_size,
+                                           int max_blocks_per_seq, int partition_tokens);
+
+/*
  * kv_cache_append - store the step's new K and V rows into their cache slots.
  *
  * For every token t < num_tokens with slot = slot_mapping[t] >= 0:

@@ -20,6 +20,8 @@ from ._lib import (  # noqa: F401
     abi_version,
     alloc_workspace,
     get_device_error,
+    gqa_partition_tokens,
+    gqa_workspace_size,
     kv_block_copy,
     kv_cache_append,
     load,

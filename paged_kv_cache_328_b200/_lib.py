@@ -37,6 +37,11 @@ SIGNATURES = {
     "pkv_get_device_error": (_c_int, [_c_void_p, ctypes.POINTER(_c_int)]),
     "pkv_strerror": (ctypes.c_char_p, [_c_int]),
     "pkv_abi_version": (_c_int, []),
+    "paged_attn_decode_gqa": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                       _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                       _c_float, _c_void_p, _c_int, _c_void_p, _c_size_t, _c_void_p]),
+    "paged_attn_decode_gqa_workspace_size": (_c_size_t, [_c_int] * 7),
+    "paged_attn_decode_gqa_partition_tokens": (_c_int, [_c_int] * 7),
     "paged_attn_decode_noalloc": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                            _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                            _c_float, _c_void_p, _c_int, _c_void_p]),
@@ -118,22 +123,42 @@ def partition_tokens(num_seqs, num_heads, head_dim, block_size, max_blocks, part
     return rc
 
 
+def gqa_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks, partition_tokens=0):
+    n = load().paged_attn_decode_gqa_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                                    max_blocks, partition_tokens)
+    if n == ctypes.c_size_t(-1).value:
+        raise PagedKVError(-1, "paged_attn_decode_gqa_workspace_size")
+    return n
+
+
+def gqa_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks, partition_tokens=0):
+    rc = load().paged_attn_decode_gqa_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                                       max_blocks, partition_tokens)
+    if rc < 0:
+        raise PagedKVError(rc, "paged_attn_decode_gqa_partition_tokens")
+    return rc
+
+
 def alloc_workspace(q, k_cache, block_tables, partition_tokens=0):
     """A uint8 workspace tensor sized for these inputs, on q's device."""
     S, H, D = q.shape
-    B = k_cache.shape[2]
-    n = workspace_size(S, H, D, B, block_tables.shape[1], partition_tokens)
+    Hkv, B = k_cache.shape[1], k_cache.shape[2]
+    n = gqa_workspace_size(S, H, Hkv, D, B, block_tables.shape[1], partition_tokens)
     return torch.empty(n, dtype=torch.uint8, device=q.device)
 
 
 def paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out=None,
                       partition_tokens=0, workspace=None, stream=None):
-    """out[s, h] = softmax(scale * K q) V over the paged context; returns out (float32 [S, H, D])."""
+    """out[s, h] = softmax(scale * K q) V over the paged context; returns out (float32 [S, H, D]).
+
+    The caches may hold fewer heads than q (grouped-query attention): with Hkv K/V
+    heads, query head h reads K/V head h // (H // Hkv).
+    """
     lib = load()
     S, H, D = q.shape
-    NB, Hc, B, Dc = k_cache.shape
-    if (Hc, Dc) != (H, D) or tuple(v_cache.shape) != tuple(k_cache.shape):
-        raise ValueError("q [S,H,D] and caches [NB,H,B,D] disagree")
+    NB, Hkv, B, Dc = k_cache.shape
+    if Dc != D or Hkv <= 0 or H % Hkv or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("q [S,H,D] and caches [NB,Hkv,B,D] disagree (H must be a multiple of Hkv)")
     if q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
         raise TypeError("q, k_cache and v_cache must share one storage dtype")
     if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.shape != (S,):
@@ -149,12 +174,15 @@ def paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale, ou
     args = (_cuda(q, "q", DTYPE_CODE), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
             _cuda(block_tables, "block_tables", (torch.int32,)),
             _cuda(context_lens, "context_lens", (torch.int32,)),
-            S, H, D, B, block_tables.shape[1], NB, dt, float(scale),
+            S, H, Hkv, D, B, block_tables.shape[1], NB, dt, float(scale),
             _cuda(out, "out", (torch.float32,)), int(partition_tokens),
             _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size())
     with torch.cuda.device(q.device):
-        rc = lib.paged_attn_decode(*args, _stream(q.device, stream))
-    _check(rc, "paged_attn_decode")
+        if Hkv == H:
+            rc = lib.paged_attn_decode(*args[:6], *args[7:], _stream(q.device, stream))
+        else:
+            rc = lib.paged_attn_decode_gqa(*args, _stream(q.device, stream))
+    _check(rc, "paged_attn_decode" if Hkv == H else "paged_attn_decode_gqa")
     return out
 
 

@@ -83,7 +83,9 @@ struct DecodeParams {
   const void* v_cache;
   const int32_t* block_tables;
   const int32_t* context_lens;
-  int num_heads;
+  int num_heads;      // query heads (Hq)
+  int num_kv_heads;   // K/V heads in the pools (Hkv); query head h reads K/V head h / group
+  int group;          // Hq / Hkv
   int block_size;
   int max_blocks;
   int num_blocks;
@@ -340,7 +342,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
         if (mine) {
           if (phys >= 0 && phys < prm.num_blocks) {
             const int rows = min(unit_rows, cur.t_end - u_t0);
-            src_off = pool_row(phys, cur.h, u_t0 % B, H, B, D);
+            src_off = pool_row(phys, cur.h / prm.group, u_t0 % B, prm.num_kv_heads, B, D);
             bytes = (uint32_t)rows * Tr::kRowBytes;
           } else {
             flag_error(PKV_DEV_BLOCK_ID);

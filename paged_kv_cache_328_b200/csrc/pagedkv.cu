@@ -10,9 +10,12 @@
 #include <cstring>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "pagedkv.h"
 #include "pkv_device.cuh"
 #include "decode.cuh"
+#include "decode_gqa.cuh"
 #include "cache_ops.cuh"
 
 namespace {
@@ -61,8 +64,12 @@ constexpr long long kRefCtas = 148 * 2;
 // (one warp, 32 sequences per step; the lengths are staged in shared memory).
 constexpr long long kSortedUnitsMax = pkv::kPlanSortMaxSeqs;
 
-int make_plan(int S, int H, int D, int B, int MB, int requested, DecodePlan* plan) {
+// H = query heads (partial states are kept per query head); Hkv = K/V heads (the
+// no-split decision counts (sequence, K/V head) pairs so that it does not depend on
+// which kernel runs).
+int make_plan(int S, int H, int Hkv, int D, int B, int MB, int requested, DecodePlan* plan) {
   if (S < 0 || H <= 0 || MB <= 0) return PKV_EINVAL;
+  if (Hkv <= 0 || H % Hkv != 0) return PKV_EINVAL;
   if (!head_dim_ok(D) || !block_size_ok(B)) return PKV_EUNSUPPORTED;
   if (S > 65535 || H > 65535) return PKV_EINVAL;
   const long long max_ctx = (long long)MB * B;
@@ -70,7 +77,7 @@ int make_plan(int S, int H, int D, int B, int MB, int requested, DecodePlan* pla
   if (requested < 0 || (requested > 0 && requested % B != 0)) return PKV_EINVAL;
   long long pt = requested;
   if (requested == 0) {
-    const bool enough_units = (long long)S * H >= 4 * kRefCtas && max_ctx <= 4096;
+    const bool enough_units = (long long)S * Hkv >= 4 * kRefCtas && max_ctx <= 4096;
     pt = (max_ctx <= kAutoPartitionTokens || enough_units) ? max_ctx : kAutoPartitionTokens;
   }
   if (pt >= max_ctx) pt = max_ctx;
@@ -176,6 +183,88 @@ int dispatch_decode(pkv_dtype dt, const pkv::DecodeParams& prm, long long max_un
   return PKV_EDTYPE;
 }
 
+// ---------------------------------------------------------------------------
+// Grouped-query tensor-core kernel: tensor maps over the pools and the launch.
+// ---------------------------------------------------------------------------
+std::mutex g_tmap_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+
+int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::lock_guard<std::mutex> lk(g_tmap_mu);
+  if (g_encode_tiled == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || p == nullptr)
+      return PKV_ECUDA;
+    g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  *fn = g_encode_tiled;
+  return PKV_OK;
+}
+
+// 2-D view of one pool: rows = num_blocks * Hkv * B, columns = D (16-bit); boxes of
+// 64 columns x box_rows rows, 128-byte swizzle.
+int encode_pool_map(CUtensorMap* map, const void* pool, long long rows, int D, int box_rows, pkv_dtype dt) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  if (tensor_map_encoder(&enc) != PKV_OK) return PKV_ECUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  const CUtensorMapDataType type =
+      dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUresult r = enc(map, type, 2, const_cast<void*>(pool), dims, strides, box, elem_strides,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ECUDA;
+}
+
+template <typename T, int D, int NS>
+int launch_gqa(const pkv::GqaParams& prm, long long max_units, cudaStream_t st) {
+  using Tr = pkv::GqaTraits<D, NS>;
+  static int occ[kMaxDevices];
+  int dev;
+  if (current_device(&dev) != PKV_OK) return PKV_ECUDA;
+  const int sms = sm_count(dev);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (occ[dev] == 0) {
+      auto kern = pkv::paged_decode_gqa_kernel<T, D, NS>;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::kSmemAlloc) != cudaSuccess)
+        return PKV_ECUDA;
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, pkv::kDecodeThreads, Tr::kSmemAlloc) !=
+              cudaSuccess ||
+          n <= 0)
+        return PKV_ECUDA;
+      occ[dev] = n;
+    }
+  }
+  if (sms <= 0) return PKV_ECUDA;
+  long long grid = (long long)sms * occ[dev];
+  if (grid > max_units) grid = max_units;
+  if (grid < 1) grid = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(pkv::kDecodeThreads);
+  cfg.dynamicSmemBytes = Tr::kSmemAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, pkv::paged_decode_gqa_kernel<T, D, NS>, prm) != cudaSuccess) return PKV_ECUDA;
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+// Whether the tensor-core grouped-query kernel serves these arguments.
+bool use_gqa_kernel(int Hq, int Hkv, int B, int NB, pkv_dtype dt) {
+  const int G = Hq / Hkv;
+  return G >= 2 && G <= pkv::kGqaRows && dt != PKV_F32 && (long long)NB * Hkv * B < (1LL << 31);
+}
+
 // The merge is a programmatic dependent of the decode kernel: its CTAs may be
 // scheduled as decode CTAs run out of units and wait for the decode to finish.
 template <int D>
@@ -213,7 +302,8 @@ extern "C" {
 size_t paged_attn_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int block_size,
                                         int max_blocks_per_seq, int partition_tokens) {
   DecodePlan plan;
-  if (make_plan(num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens, &plan) != PKV_OK)
+  if (make_plan(num_seqs, num_heads, num_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens,
+                &plan) != PKV_OK)
     return (size_t)-1;
   return plan.bytes;
 }
@@ -221,17 +311,26 @@ size_t paged_attn_decode_workspace_size(int num_seqs, int num_heads, int head_di
 int paged_attn_decode_partition_tokens(int num_seqs, int num_heads, int head_dim, int block_size,
                                        int max_blocks_per_seq, int partition_tokens) {
   DecodePlan plan;
-  const int rc = make_plan(num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens, &plan);
+  const int rc = make_plan(num_seqs, num_heads, num_heads, head_dim, block_size, max_blocks_per_seq,
+                           partition_tokens, &plan);
   return rc != PKV_OK ? rc : plan.part_tokens;
 }
 
-int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
-                      const int32_t* context_lens, int num_seqs, int num_heads, int head_dim, int block_size,
-                      int max_blocks_per_seq, int num_blocks, pkv_dtype dtype, float scale, float* out,
-                      int partition_tokens, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Paged decode for num_heads query heads over num_kv_heads K/V heads (equal for
+// multi-head attention).  Shared by every decode entry point.
+int decode_impl(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                int block_size, int max_blocks_per_seq, int num_blocks, pkv_dtype dtype, float scale, float* out,
+                int partition_tokens, void* workspace, size_t workspace_bytes, void* stream) {
   if (elem_bytes(dtype) == 0) return PKV_EDTYPE;
+  if (num_kv_heads <= 0 || num_heads <= 0 || num_heads % num_kv_heads != 0) return PKV_EINVAL;
   DecodePlan plan;
-  const int rc = make_plan(num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens, &plan);
+  const int rc = make_plan(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           partition_tokens, &plan);
   if (rc != PKV_OK) return rc;
   if (num_blocks <= 0) return PKV_EINVAL;
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return PKV_EINVAL;
@@ -259,6 +358,8 @@ int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache, c
   prm.block_tables = block_tables;
   prm.context_lens = context_lens;
   prm.num_heads = num_heads;
+  prm.num_kv_heads = num_kv_heads;
+  prm.group = num_heads / num_kv_heads;
   prm.block_size = block_size;
   prm.max_blocks = max_blocks_per_seq;
   prm.num_blocks = num_blocks;
@@ -277,8 +378,42 @@ int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache, c
       context_lens, num_seqs, max_ctx, plan.part_tokens, plan.sort ? 1 : 0,
       reinterpret_cast<uint32_t*>(ws + plan.off_units), prm.counters);
   if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
-  const long long max_units = (long long)num_seqs * num_heads * plan.max_parts;
-  if (result == PKV_OK) {
+  if (result == PKV_OK && use_gqa_kernel(num_heads, num_kv_heads, block_size, num_blocks, dtype)) {
+    static_assert(alignof(pkv::GqaParams) >= 64, "tensor maps need 64-byte alignment");
+    pkv::GqaParams g;
+    const long long rows = (long long)num_blocks * num_kv_heads * block_size;
+    const int box_rows = block_size < pkv::kGqaTile ? block_size : pkv::kGqaTile;
+    if (encode_pool_map(&g.tmap_k, k_cache, rows, head_dim, box_rows, dtype) != PKV_OK ||
+        encode_pool_map(&g.tmap_v, v_cache, rows, head_dim, box_rows, dtype) != PKV_OK) {
+      result = PKV_ECUDA;
+    } else {
+      g.q = q;
+      g.block_tables = block_tables;
+      g.context_lens = context_lens;
+      g.num_heads = num_heads;
+      g.num_kv_heads = num_kv_heads;
+      g.group = num_heads / num_kv_heads;
+      g.block_size = block_size;
+      g.max_blocks = max_blocks_per_seq;
+      g.num_blocks = num_blocks;
+      g.scale_log2 = prm.scale_log2;
+      g.part_tokens = plan.part_tokens;
+      g.max_parts = plan.max_parts;
+      g.out = out;
+      g.ws_acc = prm.ws_acc;
+      g.ws_ml = prm.ws_ml;
+      g.units = prm.units;
+      g.counters = prm.counters;
+      const long long max_units = (long long)num_seqs * num_kv_heads * plan.max_parts;
+      if (dtype == PKV_BF16)
+        result = head_dim == 64 ? launch_gqa<__nv_bfloat16, 64, 4>(g, max_units, st)
+                                : launch_gqa<__nv_bfloat16, 128, 4>(g, max_units, st);
+      else
+        result = head_dim == 64 ? launch_gqa<__half, 64, 4>(g, max_units, st)
+                                : launch_gqa<__half, 128, 4>(g, max_units, st);
+    }
+  } else if (result == PKV_OK) {
+    const long long max_units = (long long)num_seqs * num_heads * plan.max_parts;
     result = head_dim == 64 ? dispatch_decode<64>(dtype, prm, max_units, st)
                             : dispatch_decode<128>(dtype, prm, max_units, st);
   }
@@ -289,6 +424,45 @@ int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache, c
   }
   if (owned && cudaFreeAsync(ws, st) != cudaSuccess && result == PKV_OK) result = PKV_ECUDA;
   return result;
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, int num_seqs, int num_heads, int head_dim, int block_size,
+                      int max_blocks_per_seq, int num_blocks, pkv_dtype dtype, float scale, float* out,
+                      int partition_tokens, void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads, num_heads, head_dim,
+                     block_size, max_blocks_per_seq, num_blocks, dtype, scale, out, partition_tokens, workspace,
+                     workspace_bytes, stream);
+}
+
+size_t paged_attn_decode_gqa_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                            int block_size, int max_blocks_per_seq, int partition_tokens) {
+  DecodePlan plan;
+  if (make_plan(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens,
+                &plan) != PKV_OK)
+    return (size_t)-1;
+  return plan.bytes;
+}
+
+int paged_attn_decode_gqa_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                           int block_size, int max_blocks_per_seq, int partition_tokens) {
+  DecodePlan plan;
+  const int rc = make_plan(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           partition_tokens, &plan);
+  return rc != PKV_OK ? rc : plan.part_tokens;
+}
+
+int paged_attn_decode_gqa(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                          const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                          int block_size, int max_blocks_per_seq, int num_blocks, pkv_dtype dtype, float scale,
+                          float* out, int partition_tokens, void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                     block_size, max_blocks_per_seq, num_blocks, dtype, scale, out, partition_tokens, workspace,
+                     workspace_bytes, stream);
 }
 
 int kv_cache_append(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
@@ -438,7 +612,8 @@ extern "C" int paged_attn_decode_noalloc(const void* q, const void* k_cache, con
   if (need == (size_t)-1) {
     // the same argument error paged_attn_decode reports
     DecodePlan plan;
-    return make_plan(num_seqs, num_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens, &plan);
+    return make_plan(num_seqs, num_heads, num_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens,
+                     &plan);
   }
   if (need > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_EWORKSPACE;
   if (num_seqs == 0) return PKV_OK;

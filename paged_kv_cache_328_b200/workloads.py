@@ -62,6 +62,11 @@ class Workload:
     v_new: torch.Tensor
     partition_tokens: int = 0         # split-context partition size (0 = library default)
     info: dict = field(default_factory=dict)
+    Hkv: int = 0                      # K/V heads in the pools (0: same as H, multi-head)
+
+    def __post_init__(self):
+        if not self.Hkv:
+            self.Hkv = self.H
 
     # ---- sizes -------------------------------------------------------------
     @property
@@ -69,16 +74,16 @@ class Workload:
         return ELEM_BYTES[self.dtype]
 
     def kv_bytes_attended(self):
-        """K+V bytes the decode reads by definition: sum(ctx) * H * D * e * 2."""
-        return int(self.context_lens.astype(np.int64).sum()) * self.H * self.D * self.elem_bytes * 2
+        """K+V bytes the decode reads by definition: sum(ctx) * Hkv * D * e * 2."""
+        return int(self.context_lens.astype(np.int64).sum()) * self.Hkv * self.D * self.elem_bytes * 2
 
     def append_bytes(self):
         n = int((self.slot_mapping >= 0).sum())
-        return n * self.H * self.D * self.elem_bytes * 2
+        return n * self.Hkv * self.D * self.elem_bytes * 2
 
     def copy_bytes(self):
         """K+V bytes read (equal to bytes written) by the step's block copies."""
-        return len(self.cow_pairs) * self.H * self.B * self.D * self.elem_bytes * 2
+        return len(self.cow_pairs) * self.Hkv * self.B * self.D * self.elem_bytes * 2
 
     # ---- host views (raw stored elements) ------------------------------------
     def host(self, t):
@@ -131,13 +136,19 @@ def _token_coords(tables, ctx, B, device, skip_last):
 
 def build_paged(context_lens, H, D, B, dtype, seed, *, device="cpu", num_blocks=None,
                 pool_factor=1.2, max_blocks=None, preappend=False, scale=None,
-                placement_seed=None, name="custom", partition_tokens=0, logical=None):
+                placement_seed=None, name="custom", partition_tokens=0, logical=None,
+                num_q_heads=None):
     """Independent sequences with a random physical placement of their blocks.
 
+    ``H`` is the number of K/V heads in the pools; ``num_q_heads`` (default H)
+    the number of query heads, a multiple of H (grouped-query attention).
     ``logical`` may pass pre-drawn per-token rows ``(K_log, V_log, q)`` with
     ``K_log``/``V_log`` of shape ``[sum(ctx), H, D]`` so that several block sizes
     share the same token data; otherwise they are drawn from ``seed``.
     """
+    Hq = H if num_q_heads is None else int(num_q_heads)
+    if Hq % H:
+        raise ValueError("query heads must be a multiple of K/V heads")
     ctx = np.asarray(context_lens, dtype=np.int64)
     S = len(ctx)
     nblk = -(-ctx // B)
@@ -166,7 +177,7 @@ def build_paged(context_lens, H, D, B, dtype, seed, *, device="cpu", num_blocks=
     if logical is None:
         K_log = _randn((total, H, D), gen, dtype, device)
         V_log = _randn((total, H, D), gen, dtype, device)
-        q = _randn((S, H, D), gen, dtype, device)
+        q = _randn((S, Hq, D), gen, dtype, device)
     else:
         K_log, V_log, q = logical
 
@@ -197,7 +208,7 @@ def build_paged(context_lens, H, D, B, dtype, seed, *, device="cpu", num_blocks=
     v_new = V_log.index_select(0, lastt)
 
     return Workload(
-        name=name, S=S, H=H, D=D, B=B, dtype=dtype,
+        name=name, S=S, H=Hq, D=D, B=B, dtype=dtype, Hkv=H,
         scale=(1.0 / math.sqrt(D)) if scale is None else float(scale),
         num_blocks=num_blocks, max_blocks=max_blocks,
         context_lens=ctx.astype(np.int32), block_tables=tables, slot_mapping=slot,
@@ -382,6 +393,15 @@ def make_cow(device="cpu", preappend=False, groups=32, n=4, prompt=512, tail_max
     )
 
 
+def make_gqa(group, device="cpu", preappend=False, S=256, Hkv=8, B=16):
+    """Grouped-query decode layer: 8 K/V heads x 128 (bf16) shared by `group` query heads
+    each, batch 256, contexts U{1..2048} (the batch-256 layer's lengths), block size 16."""
+    seed = BASE_SEED + 10 + group
+    ctx = opt13b_lengths(S)
+    return build_paged(ctx, H=Hkv, D=128, B=B, dtype="bf16", seed=seed, device=device, preappend=preappend,
+                       max_blocks=2048 // B, num_q_heads=Hkv * group, name=f"gqa{group}_B{B}")
+
+
 def make(name, device="cpu", preappend=False, B=None):
     if name == "tiny":
         return make_tiny(device=device, preappend=preappend)
@@ -393,6 +413,8 @@ def make(name, device="cpu", preappend=False, B=None):
         return make_cow(device=device, preappend=preappend)
     if name == "longctx":
         return make_longctx(device=device, preappend=preappend)
+    if name.startswith("gqa"):
+        return make_gqa(int(name[3:]), device=device, preappend=preappend, B=16 if B is None else B)
     raise ValueError(f"unknown workload {name!r}")
 
 

@@ -25,6 +25,7 @@ class Snapshot:
 
     def __init__(self, w, s, h):
         self.s, self.h = s, h
+        kvh = h // (w.H // w.Hkv)  # K/V head read by query head h
         ctx = int(w.context_lens[s])
         nblk = -(-ctx // w.B)
         row = [int(b) for b in w.block_tables[s, :nblk]]
@@ -32,8 +33,8 @@ class Snapshot:
         blocks = sorted(set(row) | set(srcs))
         self.remap = {b: i for i, b in enumerate(blocks)}
         idx = torch.tensor(blocks, dtype=torch.long, device=w.k_pool.device)
-        self.k = w.host(w.k_pool.index_select(0, idx)[:, h:h + 1].contiguous())
-        self.v = w.host(w.v_pool.index_select(0, idx)[:, h:h + 1].contiguous())
+        self.k = w.host(w.k_pool.index_select(0, idx)[:, kvh:kvh + 1].contiguous())
+        self.v = w.host(w.v_pool.index_select(0, idx)[:, kvh:kvh + 1].contiguous())
         self.table = np.array([self.remap[b] for b in row], dtype=np.int64).reshape(1, -1)
         if nblk == 0:
             self.table = np.full((1, 1), -1, dtype=np.int64)
@@ -46,8 +47,8 @@ class Snapshot:
         else:
             self.slot = np.array([-1], dtype=np.int64)
         self.q = w.host(w.q[s:s + 1, h:h + 1].contiguous())
-        self.knew = w.host(w.k_new[s:s + 1, h:h + 1].contiguous()) if w.k_new.shape[0] > s else None
-        self.vnew = w.host(w.v_new[s:s + 1, h:h + 1].contiguous()) if w.v_new.shape[0] > s else None
+        self.knew = w.host(w.k_new[s:s + 1, kvh:kvh + 1].contiguous()) if w.k_new.shape[0] > s else None
+        self.vnew = w.host(w.v_new[s:s + 1, kvh:kvh + 1].contiguous()) if w.v_new.shape[0] > s else None
         self.ctx = ctx
 
     def expected(self, w, copy=True, append=True, ctx=None):
