@@ -71,13 +71,14 @@ struct GqaTraits {
   static constexpr int kHdrOffset = kQOffset + NS * kQBytes;
   static constexpr int kBarOffset = kHdrOffset + NS * 16;
   static constexpr int kAbortOffset = kBarOffset + (2 * NS + 1) * 8;
-  static constexpr int kRedOffset = (kAbortOffset + 16 + 127) / 128 * 128;
-  static constexpr int kRedAccFloats = kConsumerWarps * kGqaRows * D;
+  static constexpr int kRedMlOffset = (kAbortOffset + 16 + 127) / 128 * 128;
+  static constexpr int kRedAccFloats = kConsumerWarps * kGqaRows * D;  // lives in the unit's last stage
   static constexpr int kRedMlFloats = kConsumerWarps * kGqaRows * 2;
-  static constexpr int kSmemBytes = kRedOffset + (kRedAccFloats + kRedMlFloats) * 4;
+  static constexpr int kSmemBytes = kRedMlOffset + kRedMlFloats * 4;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // the base is rounded up to 1024 bytes
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(kStageBytes % 1024 == 0, "swizzled slabs stay 1024-byte aligned");
+  static_assert(kRedAccFloats * 4 <= kStageBytes, "the warps' row states fit in one stage");
 };
 
 // ---- PTX wrappers ------------------------------------------------------------
@@ -159,6 +160,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// 2^x with the hardware approximation (one MUFU instruction; relative error
+// ~2^-22; -inf gives +0, flush-to-zero).
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------------------
 // grid = min(#SMs x resident CTAs, units); block = kDecodeThreads (4 consumer warps + producer)
 // ---------------------------------------------------------------------------
@@ -173,8 +182,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
   uint64_t* epi = empty + NS;
   int4* hdr = reinterpret_cast<int4*>(smem + Tr::kHdrOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Tr::kAbortOffset);
-  float* red_acc = reinterpret_cast<float*>(smem + Tr::kRedOffset);  // [warp][row][D]
-  float* red_ml = red_acc + Tr::kRedAccFloats;                         // [warp][row][2]
+  float* red_ml = reinterpret_cast<float*>(smem + Tr::kRedMlOffset);  // [warp][row][2]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -391,27 +399,27 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
     }
 
     // ---- online softmax (base 2) per row; columns past the context are -inf ----
+    // Rows 8..15 (the second half of every fragment) are padding when G <= 8.
+    const int halves = G > 8 ? 2 : 1;
     float mt[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int tok = tok0 + nt * 8 + 2 * t4 + (c & 1);
-        const float v = (tok < n_valid) ? sacc[nt][c] * prm.scale_log2 : -INFINITY;
+        const float v = (tok < n_valid && (c >> 1) < halves) ? sacc[nt][c] * prm.scale_log2 : -INFINITY;
         sacc[nt][c] = v;
         mt[c >> 1] = fmaxf(mt[c >> 1], v);
       }
+    float alpha[2] = {1.f, 1.f};
+    float mnew[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int hrow = 0; hrow < 2; ++hrow) {
+      if (hrow >= halves) break;
       mt[hrow] = fmaxf(mt[hrow], __shfl_xor_sync(0xffffffffu, mt[hrow], 1));
       mt[hrow] = fmaxf(mt[hrow], __shfl_xor_sync(0xffffffffu, mt[hrow], 2));
-    }
-    float alpha[2];
-    float mnew[2];
-#pragma unroll
-    for (int hrow = 0; hrow < 2; ++hrow) {
       mnew[hrow] = fmaxf(m_r[hrow], mt[hrow]);
-      alpha[hrow] = (mnew[hrow] == -INFINITY) ? 1.f : exp2f(m_r[hrow] - mnew[hrow]);  // 0 when m was -inf
+      alpha[hrow] = (mnew[hrow] == -INFINITY) ? 1.f : ex2_fast(m_r[hrow] - mnew[hrow]);  // 0 when m was -inf
       m_r[hrow] = mnew[hrow];
       l_r[hrow] *= alpha[hrow];
     }
@@ -433,7 +441,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const float mm = mnew[c >> 1];
-          const float e = (mm == -INFINITY) ? 0.f : exp2f(sacc[nt][c] - mm);
+          const float e = (mm == -INFINITY) ? 0.f : ex2_fast(sacc[nt][c] - mm);
           p[nt][c] = e;
           l_r[c >> 1] += e;
         }
@@ -463,13 +471,15 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
         M::run(o[2 * i + 1], pa_lo, b[2], b[3]);
       }
     }
-    if (partial) fence_proxy_async_smem();  // generic writes above, async (TMA) writes next
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
+    if (!(flags & kTileLast)) {
+      if (partial) fence_proxy_async_smem();  // generic writes above, async (TMA) writes next
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      continue;
+    }
 
-    if (!(flags & kTileLast)) continue;
-
-    // ---- unit epilogue: the 4 warps hold disjoint tokens; merge their rows ----
+    // ---- unit epilogue: the 4 warps hold disjoint tokens; merge their rows in
+    //      the stage just consumed, then hand the stage back to the producer ----
     float lsum[2];
 #pragma unroll
     for (int hrow = 0; hrow < 2; ++hrow) {
@@ -478,8 +488,18 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
       v += __shfl_xor_sync(0xffffffffu, v, 2);
       lsum[hrow] = v;
     }
-    // (the previous unit's final merge has finished: every warp passed this barrier's
-    //  previous phase only after reading the reduction area)
+    // every warp has finished reading this stage's K and V before it is overwritten
+    __syncwarp();
+    if (lane == 0) mbar_arrive(epi);
+    if (!mbar_wait_bounded(epi, units_done & 1, abort_flag)) {
+      if (lane == 0) {
+        flag_error(PKV_DEV_WAIT_TIMEOUT);
+        *abort_flag = 1;
+      }
+      break;
+    }
+    ++units_done;
+    float* red_acc = reinterpret_cast<float*>(kt);  // [warp][row][D] over the consumed stage
 #pragma unroll
     for (int hrow = 0; hrow < 2; ++hrow) {
       const int row = gid + 8 * hrow;
@@ -517,7 +537,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) {
         const float mw = red_ml[(w * kGqaRows + row) * 2];
-        const float sc = (mx == -INFINITY) ? 0.f : exp2f(mw - mx);
+        const float sc = (mx == -INFINITY) ? 0.f : ex2_fast(mw - mx);
         L = fmaf(red_ml[(w * kGqaRows + row) * 2 + 1], sc, L);
         acc = fmaf(red_acc[(w * kGqaRows + row) * D + d], sc, acc);
       }
@@ -530,8 +550,9 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
         if (d == 0) prm.ws_ml[ws] = make_float2(mx, L);
       }
     }
-    // the reduction area is rewritten at the next unit's epilogue: wait until every
-    // consumer thread has read it (bounded, like every other wait)
+    // every consumer thread has read the states before the stage goes back to the
+    // producer; the generic writes are ordered before the next TMA writes
+    fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(epi);
     if (!mbar_wait_bounded(epi, units_done & 1, abort_flag)) {
@@ -542,6 +563,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
       break;
     }
     ++units_done;
+    if (lane == 0) mbar_arrive(&empty[stage]);
   }
 }
 

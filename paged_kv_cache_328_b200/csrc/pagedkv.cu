@@ -406,11 +406,11 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const i
       g.counters = prm.counters;
       const long long max_units = (long long)num_seqs * num_kv_heads * plan.max_parts;
       if (dtype == PKV_BF16)
-        result = head_dim == 64 ? launch_gqa<__nv_bfloat16, 64, 4>(g, max_units, st)
-                                : launch_gqa<__nv_bfloat16, 128, 4>(g, max_units, st);
+        result = head_dim == 64 ? launch_gqa<__nv_bfloat16, 64, 3>(g, max_units, st)
+                                : launch_gqa<__nv_bfloat16, 128, 3>(g, max_units, st);
       else
-        result = head_dim == 64 ? launch_gqa<__half, 64, 4>(g, max_units, st)
-                                : launch_gqa<__half, 128, 4>(g, max_units, st);
+        result = head_dim == 64 ? launch_gqa<__half, 64, 3>(g, max_units, st)
+                                : launch_gqa<__half, 128, 3>(g, max_units, st);
     }
   } else if (result == PKV_OK) {
     const long long max_units = (long long)num_seqs * num_heads * plan.max_parts;
