@@ -40,6 +40,7 @@ from .paged_attention import (
     softmax_weights,
     paged_decode,
     paged_decode_selected,
+    paged_multi_query,
 )
 from .cache_ops import kv_append, kv_block_copy, gather_kv
 
@@ -51,6 +52,7 @@ __all__ = [
     "softmax_weights",
     "paged_decode",
     "paged_decode_selected",
+    "paged_multi_query",
     "kv_append",
     "kv_block_copy",
     "gather_kv",

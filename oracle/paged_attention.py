@@ -28,6 +28,11 @@ Readings where the pages are silent:
   related-work list as an orthogonal way to shrink the KV cache): with Hq query
   heads and Hkv K/V heads, G = Hq / Hkv consecutive query heads share one K/V head,
   query head h reading K/V head h // G.  Hkv = Hq is ordinary multi-head attention.
+* Several query tokens per sequence (a prefill chunk appended to a cached prefix,
+  or draft tokens checked in one pass; the video summary's "주요 인사이트" names
+  chunked prefill and speculative decoding): the Lq new tokens are the last Lq of
+  the context, and query token j (0-based) attends the positions before and at its
+  own, i.e. the first ctx - Lq + j + 1 tokens.  Lq = 1 is decode.
 """
 
 import numpy as np
@@ -113,3 +118,26 @@ def paged_decode(q, k_pool, v_pool, block_tables, context_lens, scale, block_siz
     flat = paged_decode_selected(q, k_pool, v_pool, block_tables, context_lens, scale,
                                  block_size, dtype, sel)
     return flat.reshape(S, H, D)
+
+
+def paged_multi_query(q, k_pool, v_pool, block_tables, context_lens, scale, block_size, dtype):
+    """Outputs for Lq query tokens per sequence: float64 ``[S, Lq, Hq, D]``.
+
+    ``q`` is ``[S, Lq, Hq, D]``; the context of sequence s (``context_lens[s]``
+    tokens) already holds the Lq new tokens as its last Lq positions, and query
+    token j attends the first ``context_lens[s] - Lq + j + 1`` tokens (none when
+    that count is not positive).
+    """
+    S, Lq, Hq, D = q.shape
+    Hkv = k_pool.shape[1]
+    group = Hq // Hkv
+    out = np.zeros((S, Lq, Hq, D), dtype=np.float64)
+    for s in range(S):
+        ctx = int(context_lens[s])
+        for j in range(Lq):
+            visible = max(0, ctx - Lq + j + 1)
+            for h in range(Hq):
+                K = to_f64(gather_rows(k_pool, block_tables[s], visible, h // group, block_size), dtype)
+                V = to_f64(gather_rows(v_pool, block_tables[s], visible, h // group, block_size), dtype)
+                out[s, j, h] = attend(to_f64(q[s, j, h], dtype), K, V, scale)
+    return out

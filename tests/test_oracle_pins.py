@@ -463,6 +463,48 @@ def check_gqa_equals_replicated_mha():
         assert np.max(np.abs(gqa[0] - ref.numpy())) <= 1e-12
 
 
+def check_multi_query_rows_are_shorter_decodes():
+    """Query token j of Lq sees the first ctx - Lq + j + 1 tokens: each row equals the
+    decode oracle over that shorter context, and the last row equals decode over ctx."""
+    rng = np.random.default_rng(23)
+    Hq, Hkv, D, B, nb = 4, 2, 64, 16, 14
+    for dtype in ("f16", "bf16"):
+        ctxs = [7, 40, 3]
+        Lq = 5
+        tables = []
+        perm = rng.permutation(nb)
+        cur = 0
+        for c in ctxs:
+            n = -(-c // B)
+            tables.append([int(x) for x in perm[cur:cur + n]] + [-1] * (3 - n))
+            cur += n
+        kp = random_stored(rng, (nb, Hkv, B, D), dtype)
+        vp = random_stored(rng, (nb, Hkv, B, D), dtype)
+        q = random_stored(rng, (len(ctxs), Lq, Hq, D), dtype)
+        got = oracle.paged_multi_query(q, kp, vp, np.array(tables), np.array(ctxs), 0.125, B, dtype)
+        for s, c in enumerate(ctxs):
+            for j in range(Lq):
+                vis = max(0, c - Lq + j + 1)
+                dec = oracle.paged_decode(q[s:s + 1, j], kp, vp, np.array([tables[s]]), np.array([vis]),
+                                          0.125, B, dtype)[0]
+                assert np.array_equal(got[s, j], dec), (s, j)
+        # brute force for one row of a sequence whose context is longer than Lq
+        s, j, h = 1, 2, 3
+        vis = ctxs[s] - Lq + j + 1
+        qv = storage_lib(q[s, j, h], dtype)
+        logits, rows = [], []
+        for t in range(vis):
+            blk, off = tables[s][t // B], t % B
+            kr = storage_lib(kp[blk, h // (Hq // Hkv), off], dtype)
+            rows.append(storage_lib(vp[blk, h // (Hq // Hkv), off], dtype))
+            logits.append(0.125 * math.fsum(float(qv[d]) * float(kr[d]) for d in range(D)))
+        m = max(logits)
+        e = [math.exp(x - m) for x in logits]
+        z = math.fsum(e)
+        want = [math.fsum(e[t] * float(rows[t][d]) for t in range(vis)) / z for d in range(D)]
+        assert np.max(np.abs(got[s, j, h] - np.array(want))) <= 1e-12
+
+
 def all_pin_checks(golden_dir):
     return [
         check_storage_f16,
@@ -484,6 +526,7 @@ def all_pin_checks(golden_dir):
         check_append_brute_force,
         check_block_copy_brute_force,
         check_gqa_equals_replicated_mha,
+        check_multi_query_rows_are_shorter_decodes,
     ]
 
 
@@ -558,6 +601,10 @@ def test_block_copy_brute_force():
 
 def test_gqa_equals_replicated_mha():
     check_gqa_equals_replicated_mha()
+
+
+def test_multi_query_rows_are_shorter_decodes():
+    check_multi_query_rows_are_shorter_decodes()
 
 
 def test_softmax_weights_sum_to_one():
