@@ -176,6 +176,34 @@ int paged_attn_decode_gqa_partition_tokens(int num_seqs, int num_heads, int num_
                                            int max_blocks_per_seq, int partition_tokens);
 
 /*
+ * paged_attn_multi_query - several query tokens per sequence over its paged context.
+ *
+ * For a prefill chunk appended to a cached prefix, or draft tokens checked in one
+ * pass (the video summary "KV 캐시·PagedAttention로 LLM 추론 속도와 GPU 처리량 높이기",
+ * "주요 인사이트": chunked prefill, speculative decoding).  The q_len new tokens are
+ * already in the cache as the last q_len of the context_lens[s] tokens; query token
+ * j (0-based) of sequence s attends the first context_lens[s] - q_len + j + 1
+ * tokens (causal), or none when that count is not positive (its row is zero).
+ * num_heads query heads share num_kv_heads K/V heads as in paged_attn_decode_gqa.
+ *
+ *   q             [num_seqs][q_len][num_heads][head_dim], fp16 or bf16.
+ *   out           float32 [num_seqs][q_len][num_heads][head_dim].
+ *   The rest is as in paged_attn_decode_gqa; fp32 storage returns PKV_EUNSUPPORTED.
+ *   q_len = 1 computes exactly what paged_attn_decode_gqa computes.
+ */
+int paged_attn_multi_query(const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens,
+                           int num_seqs, int q_len, int num_heads, int num_kv_heads,
+                           int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                           pkv_dtype dtype, float scale, float* out, int partition_tokens,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes paged_attn_multi_query needs; (size_t)-1 for rejected arguments. */
+size_t paged_attn_multi_query_workspace_size(int num_seqs, int q_len, int num_heads,
+                                             int num_kv_heads, int head_dim, int block_size,
+                                             int max_blocks_per_seq, int partition_tokens);
+
+/*
  * kv_cache_append - store the step's new K and V rows into their cache slots.
  *
  * For every token t < num_tokens with slot = slot_mapping[t] >= 0:

@@ -26,6 +26,7 @@ from ._lib import (  # noqa: F401
     kv_cache_append,
     load,
     paged_attn_decode,
+    paged_attn_multi_query,
     paged_kv_gather,
     partition_tokens,
     strerror,

@@ -42,6 +42,9 @@ SIGNATURES = {
                                        _c_float, _c_void_p, _c_int, _c_void_p, _c_size_t, _c_void_p]),
     "paged_attn_decode_gqa_workspace_size": (_c_size_t, [_c_int] * 7),
     "paged_attn_decode_gqa_partition_tokens": (_c_int, [_c_int] * 7),
+    "paged_attn_multi_query": (_c_int, [_c_void_p] * 5 + [_c_int] * 9 + [_c_float, _c_void_p, _c_int, _c_void_p,
+                                                                     _c_size_t, _c_void_p]),
+    "paged_attn_multi_query_workspace_size": (_c_size_t, [_c_int] * 8),
     "paged_attn_decode_noalloc": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                            _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                            _c_float, _c_void_p, _c_int, _c_void_p]),
@@ -280,4 +283,38 @@ def paged_attn_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, s
     with torch.cuda.device(q.device):
         rc = lib.paged_attn_decode_noalloc(*args, _stream(q.device, stream))
     _check(rc, "paged_attn_decode_noalloc")
+    return out
+
+
+def paged_attn_multi_query(q, k_cache, v_cache, block_tables, context_lens, scale, out=None,
+                           partition_tokens=0, workspace=None, stream=None):
+    """Several query tokens per sequence: q [S, Lq, H, D] -> out float32 [S, Lq, H, D].
+
+    The Lq new tokens are the last Lq positions of each context (already appended);
+    query token j attends the first ctx - Lq + j + 1 tokens.
+    """
+    lib = load()
+    S, Lq, H, D = q.shape
+    NB, Hkv, B, Dc = k_cache.shape
+    if Dc != D or H % Hkv or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("q [S,Lq,H,D] and caches [NB,Hkv,B,D] disagree")
+    if q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise TypeError("q, k_cache and v_cache must share one storage dtype")
+    _cuda(q, "q", DTYPE_CODE)
+    if out is None:
+        out = torch.empty((S, Lq, H, D), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = lib.paged_attn_multi_query_workspace_size(S, Lq, H, Hkv, D, B, block_tables.shape[1], partition_tokens)
+        if n == ctypes.c_size_t(-1).value:
+            raise PagedKVError(-1, "paged_attn_multi_query_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    args = (_cuda(q, "q", DTYPE_CODE), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+            _cuda(block_tables, "block_tables", (torch.int32,)),
+            _cuda(context_lens, "context_lens", (torch.int32,)),
+            S, Lq, H, Hkv, D, B, block_tables.shape[1], NB, DTYPE_CODE[k_cache.dtype], float(scale),
+            _cuda(out, "out", (torch.float32,)), int(partition_tokens),
+            _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size())
+    with torch.cuda.device(q.device):
+        rc = lib.paged_attn_multi_query(*args, _stream(q.device, stream))
+    _check(rc, "paged_attn_multi_query")
     return out

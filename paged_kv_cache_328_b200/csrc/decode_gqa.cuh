@@ -47,6 +47,9 @@ struct GqaParams {
   int num_heads;     // Hq
   int num_kv_heads;  // Hkv
   int group;         // G = Hq / Hkv
+  int q_len;         // Lq query tokens per sequence (1 = decode)
+  int rows;          // Lq * G query rows per (sequence, K/V head); row r = (token r / G, head r % G)
+  int row_tiles;     // ceil(rows / 16)
   int block_size;
   int max_blocks;
   int num_blocks;
@@ -68,8 +71,8 @@ struct GqaTraits {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kQBytes = kGqaRows * D * 2;            // query rows of a unit
   static constexpr int kQOffset = NS * kStageBytes;
-  static constexpr int kHdrOffset = kQOffset + NS * kQBytes;
-  static constexpr int kBarOffset = kHdrOffset + NS * 16;
+  static constexpr int kHdrOffset = kQOffset + NS * kQBytes;   // NS x 2 int4 headers
+  static constexpr int kBarOffset = kHdrOffset + NS * 32;
   static constexpr int kAbortOffset = kBarOffset + (2 * NS + 1) * 8;
   static constexpr int kRedMlOffset = (kAbortOffset + 16 + 127) / 128 * 128;
   static constexpr int kRedAccFloats = kConsumerWarps * kGqaRows * D;  // lives in the unit's last stage
@@ -168,6 +171,11 @@ __device__ __forceinline__ float ex2_fast(float x) {
   return y;
 }
 
+// A unit as the producer sees it: (sequence, K/V head, 16-row tile, partition).
+struct GqaUnit {
+  int s, kvh, rt, p, t_begin, t_end, n_parts, ctx;
+};
+
 // ---------------------------------------------------------------------------
 // grid = min(#SMs x resident CTAs, units); block = kDecodeThreads (4 consumer warps + producer)
 // ---------------------------------------------------------------------------
@@ -180,7 +188,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Tr::kBarOffset);
   uint64_t* empty = full + NS;
   uint64_t* epi = empty + NS;
-  int4* hdr = reinterpret_cast<int4*>(smem + Tr::kHdrOffset);
+  int4* hdr = reinterpret_cast<int4*>(smem + Tr::kHdrOffset);  // [stage][2]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Tr::kAbortOffset);
   float* red_ml = reinterpret_cast<float*>(smem + Tr::kRedMlOffset);  // [warp][row][2]
 
@@ -189,6 +197,8 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
   const int Hq = prm.num_heads;
   const int Hkv = prm.num_kv_heads;
   const int G = prm.group;
+  const int Lq = prm.q_len;
+  const int RT = prm.row_tiles;
   const int max_ctx = prm.max_blocks * prm.block_size;
   const int PT = prm.part_tokens;
 
@@ -216,20 +226,23 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
     const int B = prm.block_size;
     const int unit_rows = min(B, kGqaTile);
     const int units_per_tile = kGqaTile / unit_rows;
-    const long long total_units = (long long)prm.counters[1] * Hkv;
-    const uint32_t q_bytes = (uint32_t)(G * D * 2);
+    const int per_sp = Hkv * RT;  // units per (sequence, partition)
+    const long long total_units = (long long)prm.counters[1] * per_sp;
+    const uint32_t row_bytes = (uint32_t)(D * 2);
     const uint32_t run_bytes = (uint32_t)(unit_rows * 128);  // one 64-column box
 
     auto describe = [&](int u, uint32_t sp) {
-      UnitDesc d{0, 0, 0, 0, 0, 1};
+      GqaUnit d{0, 0, 0, 0, 0, 0, 1, 0};
       if ((long long)u < total_units) {
         d.s = (int)(sp >> 16);
         d.p = (int)(sp & 0xffffu);
-        d.h = u - (u / Hkv) * Hkv;  // K/V head
-        const int ctx = clamp_ctx(prm.context_lens[d.s], max_ctx);
+        const int rem = u - (u / per_sp) * per_sp;
+        d.kvh = rem / RT;
+        d.rt = rem - d.kvh * RT;
+        d.ctx = clamp_ctx(prm.context_lens[d.s], max_ctx);
         d.t_begin = d.p * PT;
-        d.t_end = min(ctx, d.t_begin + PT);
-        d.n_parts = parts_of(ctx, PT);
+        d.t_end = min(d.ctx, d.t_begin + PT);
+        d.n_parts = parts_of(d.ctx, PT);
       }
       return d;
     };
@@ -237,7 +250,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
     int u = 0;
     if (lane == 0) u = atomicAdd(&prm.counters[0], 1);
     u = __shfl_sync(0xffffffffu, u, 0);
-    UnitDesc cur = describe(u, (long long)u < total_units ? prm.units[u / Hkv] : 0u);
+    GqaUnit cur = describe(u, (long long)u < total_units ? prm.units[u / per_sp] : 0u);
     int it = 0;
     bool stop = false;
     while (!stop) {
@@ -278,16 +291,20 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
         }
         const unsigned loads = __ballot_sync(0xffffffffu, load);
         const bool load_q = (i == 0) && n_tok > 0;
+        const int nr = min(kGqaRows, prm.rows - cur.rt * kGqaRows);  // real query rows of this tile
         if (lane == 0) {
           const int flags = done ? kTileEnd : ((i == 0 ? kTileFirst : 0) | (i == n_tiles - 1 ? kTileLast : 0));
-          hdr[stage] = make_int4(cur.s, cur.h, cur.p | (cur.n_parts << 16), n_valid | (flags << 16));
-          const uint32_t tx = (uint32_t)__popc(loads) * 2u * Tr::kHalves * run_bytes + (load_q ? q_bytes : 0u);
+          hdr[2 * stage] = make_int4(cur.s, cur.kvh | (cur.rt << 16), cur.p | (cur.n_parts << 16),
+                                     n_valid | (flags << 16));
+          hdr[2 * stage + 1] = make_int4(tile_t0, cur.ctx, 0, 0);
+          const uint32_t tx = (uint32_t)__popc(loads) * 2u * Tr::kHalves * run_bytes +
+                              (load_q ? (uint32_t)nr * row_bytes : 0u);
           mbar_arrive_expect_tx(&full[stage], tx);
         }
         __syncwarp();
         if (load) {
           // rows of this (block, K/V head) run in the 2-D view: ((phys * Hkv + kvh) * B + offset)
-          const int y = (phys * Hkv + cur.h) * B + (u_t0 % B);
+          const int y = (phys * Hkv + cur.kvh) * B + (u_t0 % B);
           unsigned char* kt = smem + stage * Tr::kStageBytes + lane * unit_rows * 128;
 #pragma unroll
           for (int hf = 0; hf < Tr::kHalves; ++hf) {
@@ -295,13 +312,16 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
             tma_load_2d(kt + Tr::kTileBytes + hf * Tr::kSlabBytes, &prm.tmap_v, hf * 64, y, &full[stage], policy);
           }
         }
-        if (load_q && lane == 0) {
-          bulk_load(smem + Tr::kQOffset + stage * Tr::kQBytes, qg + ((size_t)cur.s * Hq + (size_t)cur.h * G) * D,
-                    q_bytes, &full[stage], policy);
+        if (load_q && lane < nr) {  // query row r = (token r / G, head-in-group r % G)
+          const int r = cur.rt * kGqaRows + lane;
+          const int tq = r / G;
+          const size_t src = (((size_t)cur.s * Lq + tq) * Hq + (size_t)cur.kvh * G + (r - tq * G)) * D;
+          bulk_load(smem + Tr::kQOffset + stage * Tr::kQBytes + lane * row_bytes, qg + src, row_bytes, &full[stage],
+                    policy);
         }
         if (i == 0 && !done) {
           u_next = __shfl_sync(0xffffffffu, u_next, 0);
-          if ((long long)u_next < total_units) sp_next = __ldcg(prm.units + u_next / Hkv);
+          if ((long long)u_next < total_units) sp_next = __ldcg(prm.units + u_next / per_sp);
         }
       }
       if (done || stop) break;
@@ -348,12 +368,23 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
       }
       break;
     }
-    const int4 hd = hdr[stage];
+    const int4 hd = hdr[2 * stage];
+    const int4 hd2 = hdr[2 * stage + 1];
     const int flags = hd.w >> 16;
     const int n_valid = hd.w & 0xffff;
     if (flags & kTileEnd) break;
     unsigned char* kt = smem + stage * Tr::kStageBytes;
     unsigned char* vt = kt + Tr::kTileBytes;
+    const int rt = hd.y >> 16;
+    const int nr = min(kGqaRows, prm.rows - rt * kGqaRows);  // real rows of this unit's tile
+    // causal limit of rows gid and gid + 8: query token tq sees positions < ctx - Lq + tq + 1
+    int lim[2];
+#pragma unroll
+    for (int hrow = 0; hrow < 2; ++hrow) {
+      const int rho = gid + 8 * hrow;
+      const int tq = (rt * kGqaRows + rho) / G;
+      lim[hrow] = rho < nr ? min(n_valid, hd2.y - Lq + tq + 1 - hd2.x) : 0;
+    }
 
     if (flags & kTileFirst) {
 #pragma unroll
@@ -398,16 +429,16 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
       }
     }
 
-    // ---- online softmax (base 2) per row; columns past the context are -inf ----
-    // Rows 8..15 (the second half of every fragment) are padding when G <= 8.
-    const int halves = G > 8 ? 2 : 1;
+    // ---- online softmax (base 2) per row; columns a row may not see are -inf ----
+    // Rows 8..15 (the second half of every fragment) are padding when nr <= 8.
+    const int halves = nr > 8 ? 2 : 1;
     float mt[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int tok = tok0 + nt * 8 + 2 * t4 + (c & 1);
-        const float v = (tok < n_valid && (c >> 1) < halves) ? sacc[nt][c] * prm.scale_log2 : -INFINITY;
+        const float v = (tok < lim[c >> 1] && (c >> 1) < halves) ? sacc[nt][c] * prm.scale_log2 : -INFINITY;
         sacc[nt][c] = v;
         mt[c >> 1] = fmaxf(mt[c >> 1], v);
       }
@@ -503,7 +534,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
 #pragma unroll
     for (int hrow = 0; hrow < 2; ++hrow) {
       const int row = gid + 8 * hrow;
-      if (row < G) {
+      if (row < nr) {
         float* dst = red_acc + (warp * kGqaRows + row) * D;
 #pragma unroll
         for (int j = 0; j < DT; ++j) {
@@ -526,10 +557,12 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
       break;
     }
     ++units_done;
-    const int us = hd.x, ukv = hd.y, up = hd.z & 0xffff, un = hd.z >> 16;
-    for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
+    const int us = hd.x, ukv = hd.y & 0xffff, up = hd.z & 0xffff, un = hd.z >> 16;
+    for (int idx = threadIdx.x; idx < nr * D; idx += kConsumerWarps * 32) {
       const int row = idx / D;
       const int d = idx - row * D;
+      const int r = rt * kGqaRows + row;
+      const int tq = r / G;
       float mx = -INFINITY;
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, red_ml[(w * kGqaRows + row) * 2]);
@@ -541,7 +574,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
         L = fmaf(red_ml[(w * kGqaRows + row) * 2 + 1], sc, L);
         acc = fmaf(red_acc[(w * kGqaRows + row) * D + d], sc, acc);
       }
-      const size_t sh = (size_t)us * Hq + (size_t)ukv * G + row;
+      const size_t sh = ((size_t)us * Lq + tq) * Hq + (size_t)ukv * G + (r - tq * G);
       if (un == 1) {
         prm.out[sh * D + d] = (L > 0.f) ? acc / L : 0.f;
       } else {

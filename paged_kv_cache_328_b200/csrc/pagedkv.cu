@@ -64,12 +64,12 @@ constexpr long long kRefCtas = 148 * 2;
 // (one warp, 32 sequences per step; the lengths are staged in shared memory).
 constexpr long long kSortedUnitsMax = pkv::kPlanSortMaxSeqs;
 
-// H = query heads (partial states are kept per query head); Hkv = K/V heads (the
-// no-split decision counts (sequence, K/V head) pairs so that it does not depend on
-// which kernel runs).
+// H = partial-state rows per sequence (query heads x query tokens); Hkv = work
+// units per (sequence, partition) counted by the no-split decision (K/V heads, so
+// that the decision does not depend on which kernel runs).
 int make_plan(int S, int H, int Hkv, int D, int B, int MB, int requested, DecodePlan* plan) {
   if (S < 0 || H <= 0 || MB <= 0) return PKV_EINVAL;
-  if (Hkv <= 0 || H % Hkv != 0) return PKV_EINVAL;
+  if (Hkv <= 0) return PKV_EINVAL;
   if (!head_dim_ok(D) || !block_size_ok(B)) return PKV_EUNSUPPORTED;
   if (S > 65535 || H > 65535) return PKV_EINVAL;
   const long long max_ctx = (long long)MB * B;
@@ -265,6 +265,47 @@ bool use_gqa_kernel(int Hq, int Hkv, int B, int NB, pkv_dtype dt) {
   return G >= 2 && G <= pkv::kGqaRows && dt != PKV_F32 && (long long)NB * Hkv * B < (1LL << 31);
 }
 
+// Launch the tensor-core kernel for Lq query tokens per sequence over the plan's
+// unit list (the plan kernel has been launched already).
+int launch_tensor_core(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                       const int32_t* context_lens, int num_seqs, int q_len, int num_heads, int num_kv_heads,
+                       int head_dim, int block_size, int max_blocks_per_seq, int num_blocks, pkv_dtype dtype,
+                       float scale_log2, float* out, const DecodePlan& plan, const pkv::DecodeParams& prm,
+                       cudaStream_t st) {
+  static_assert(alignof(pkv::GqaParams) >= 64, "tensor maps need 64-byte alignment");
+  pkv::GqaParams g;
+  const long long rows = (long long)num_blocks * num_kv_heads * block_size;
+  const int box_rows = block_size < pkv::kGqaTile ? block_size : pkv::kGqaTile;
+  if (encode_pool_map(&g.tmap_k, k_cache, rows, head_dim, box_rows, dtype) != PKV_OK ||
+      encode_pool_map(&g.tmap_v, v_cache, rows, head_dim, box_rows, dtype) != PKV_OK)
+    return PKV_ECUDA;
+  g.q = q;
+  g.block_tables = block_tables;
+  g.context_lens = context_lens;
+  g.num_heads = num_heads;
+  g.num_kv_heads = num_kv_heads;
+  g.group = num_heads / num_kv_heads;
+  g.q_len = q_len;
+  g.rows = q_len * g.group;
+  g.row_tiles = (g.rows + pkv::kGqaRows - 1) / pkv::kGqaRows;
+  g.block_size = block_size;
+  g.max_blocks = max_blocks_per_seq;
+  g.num_blocks = num_blocks;
+  g.scale_log2 = scale_log2;
+  g.part_tokens = plan.part_tokens;
+  g.max_parts = plan.max_parts;
+  g.out = out;
+  g.ws_acc = prm.ws_acc;
+  g.ws_ml = prm.ws_ml;
+  g.units = prm.units;
+  g.counters = prm.counters;
+  const long long max_units = (long long)num_seqs * num_kv_heads * g.row_tiles * plan.max_parts;
+  if (dtype == PKV_BF16)
+    return head_dim == 64 ? launch_gqa<__nv_bfloat16, 64, 3>(g, max_units, st)
+                          : launch_gqa<__nv_bfloat16, 128, 3>(g, max_units, st);
+  return head_dim == 64 ? launch_gqa<__half, 64, 3>(g, max_units, st) : launch_gqa<__half, 128, 3>(g, max_units, st);
+}
+
 // The merge is a programmatic dependent of the decode kernel: its CTAs may be
 // scheduled as decode CTAs run out of units and wait for the decode to finish.
 template <int D>
@@ -379,39 +420,9 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const i
       reinterpret_cast<uint32_t*>(ws + plan.off_units), prm.counters);
   if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
   if (result == PKV_OK && use_gqa_kernel(num_heads, num_kv_heads, block_size, num_blocks, dtype)) {
-    static_assert(alignof(pkv::GqaParams) >= 64, "tensor maps need 64-byte alignment");
-    pkv::GqaParams g;
-    const long long rows = (long long)num_blocks * num_kv_heads * block_size;
-    const int box_rows = block_size < pkv::kGqaTile ? block_size : pkv::kGqaTile;
-    if (encode_pool_map(&g.tmap_k, k_cache, rows, head_dim, box_rows, dtype) != PKV_OK ||
-        encode_pool_map(&g.tmap_v, v_cache, rows, head_dim, box_rows, dtype) != PKV_OK) {
-      result = PKV_ECUDA;
-    } else {
-      g.q = q;
-      g.block_tables = block_tables;
-      g.context_lens = context_lens;
-      g.num_heads = num_heads;
-      g.num_kv_heads = num_kv_heads;
-      g.group = num_heads / num_kv_heads;
-      g.block_size = block_size;
-      g.max_blocks = max_blocks_per_seq;
-      g.num_blocks = num_blocks;
-      g.scale_log2 = prm.scale_log2;
-      g.part_tokens = plan.part_tokens;
-      g.max_parts = plan.max_parts;
-      g.out = out;
-      g.ws_acc = prm.ws_acc;
-      g.ws_ml = prm.ws_ml;
-      g.units = prm.units;
-      g.counters = prm.counters;
-      const long long max_units = (long long)num_seqs * num_kv_heads * plan.max_parts;
-      if (dtype == PKV_BF16)
-        result = head_dim == 64 ? launch_gqa<__nv_bfloat16, 64, 3>(g, max_units, st)
-                                : launch_gqa<__nv_bfloat16, 128, 3>(g, max_units, st);
-      else
-        result = head_dim == 64 ? launch_gqa<__half, 64, 3>(g, max_units, st)
-                                : launch_gqa<__half, 128, 3>(g, max_units, st);
-    }
+    result = launch_tensor_core(q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1, num_heads,
+                                num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, dtype, prm.scale_log2,
+                                out, plan, prm, st);
   } else if (result == PKV_OK) {
     const long long max_units = (long long)num_seqs * num_heads * plan.max_parts;
     result = head_dim == 64 ? dispatch_decode<64>(dtype, prm, max_units, st)
@@ -421,6 +432,72 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const i
     result = head_dim == 64
                  ? launch_merge<64>(context_lens, num_seqs, num_heads, max_ctx, plan, prm.ws_acc, prm.ws_ml, out, st)
                  : launch_merge<128>(context_lens, num_seqs, num_heads, max_ctx, plan, prm.ws_acc, prm.ws_ml, out, st);
+  }
+  if (owned && cudaFreeAsync(ws, st) != cudaSuccess && result == PKV_OK) result = PKV_ECUDA;
+  return result;
+}
+
+// Several query tokens per sequence (tensor-core kernel only: 16-bit K/V).
+int multi_query_plan(int num_seqs, int q_len, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                     int max_blocks_per_seq, int partition_tokens, DecodePlan* plan) {
+  if (q_len <= 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0) return PKV_EINVAL;
+  const long long rows = (long long)q_len * (num_heads / num_kv_heads);
+  const long long row_tiles = (rows + pkv::kGqaRows - 1) / pkv::kGqaRows;
+  if (row_tiles > 32767 || (long long)q_len * num_heads > 65535) return PKV_EINVAL;
+  return make_plan(num_seqs, q_len * num_heads, (int)(num_kv_heads * row_tiles), head_dim, block_size,
+                   max_blocks_per_seq, partition_tokens, plan);
+}
+
+int multi_query_impl(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                     const int32_t* context_lens, int num_seqs, int q_len, int num_heads, int num_kv_heads,
+                     int head_dim, int block_size, int max_blocks_per_seq, int num_blocks, pkv_dtype dtype,
+                     float scale, float* out, int partition_tokens, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  if (elem_bytes(dtype) == 0) return PKV_EDTYPE;
+  if (dtype == PKV_F32) return PKV_EUNSUPPORTED;
+  DecodePlan plan;
+  const int rc = multi_query_plan(num_seqs, q_len, num_heads, num_kv_heads, head_dim, block_size,
+                                  max_blocks_per_seq, partition_tokens, &plan);
+  if (rc != PKV_OK) return rc;
+  if (num_blocks <= 0) return PKV_EINVAL;
+  if ((long long)num_blocks * num_kv_heads * block_size >= (1LL << 31)) return PKV_EINVAL;
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return PKV_EINVAL;
+  if (num_seqs == 0) return PKV_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PKV_EINVAL;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return PKV_EALIGN;
+  if (workspace && (!aligned(workspace, 16) || workspace_bytes < plan.bytes)) {
+    return aligned(workspace, 16) ? PKV_EWORKSPACE : PKV_EALIGN;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  bool owned = false;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (!ws) {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), plan.bytes, st) != cudaSuccess) return PKV_ECUDA;
+    owned = true;
+  }
+  pkv::DecodeParams prm = {};
+  prm.ws_acc = plan.split ? reinterpret_cast<float*>(ws + plan.off_acc) : nullptr;
+  prm.ws_ml = plan.split ? reinterpret_cast<float2*>(ws + plan.off_ml) : nullptr;
+  prm.units = reinterpret_cast<const uint32_t*>(ws + plan.off_units);
+  prm.counters = reinterpret_cast<int*>(ws);
+  const int max_ctx = max_blocks_per_seq * block_size;
+  int result = PKV_OK;
+  pkv::paged_decode_plan_kernel<<<1, pkv::kPlanThreads, 0, st>>>(
+      context_lens, num_seqs, max_ctx, plan.part_tokens, plan.sort ? 1 : 0,
+      reinterpret_cast<uint32_t*>(ws + plan.off_units), prm.counters);
+  if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
+  if (result == PKV_OK)
+    result = launch_tensor_core(q, k_cache, v_cache, block_tables, context_lens, num_seqs, q_len, num_heads,
+                                num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, dtype,
+                                scale * pkv::kLog2e, out, plan, prm, st);
+  if (result == PKV_OK && plan.split) {
+    // partial states are kept per (sequence, query token, query head): q_len * num_heads rows per sequence
+    result = head_dim == 64 ? launch_merge<64>(context_lens, num_seqs, q_len * num_heads, max_ctx, plan, prm.ws_acc,
+                                               prm.ws_ml, out, st)
+                            : launch_merge<128>(context_lens, num_seqs, q_len * num_heads, max_ctx, plan,
+                                                prm.ws_acc, prm.ws_ml, out, st);
   }
   if (owned && cudaFreeAsync(ws, st) != cudaSuccess && result == PKV_OK) result = PKV_ECUDA;
   return result;
@@ -446,6 +523,26 @@ size_t paged_attn_decode_gqa_workspace_size(int num_seqs, int num_heads, int num
                 &plan) != PKV_OK)
     return (size_t)-1;
   return plan.bytes;
+}
+
+size_t paged_attn_multi_query_workspace_size(int num_seqs, int q_len, int num_heads, int num_kv_heads,
+                                             int head_dim, int block_size, int max_blocks_per_seq,
+                                             int partition_tokens) {
+  DecodePlan plan;
+  if (multi_query_plan(num_seqs, q_len, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                       partition_tokens, &plan) != PKV_OK)
+    return (size_t)-1;
+  return plan.bytes;
+}
+
+int paged_attn_multi_query(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                           const int32_t* context_lens, int num_seqs, int q_len, int num_heads, int num_kv_heads,
+                           int head_dim, int block_size, int max_blocks_per_seq, int num_blocks, pkv_dtype dtype,
+                           float scale, float* out, int partition_tokens, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  return multi_query_impl(q, k_cache, v_cache, block_tables, context_lens, num_seqs, q_len, num_heads, num_kv_heads,
+                          head_dim, block_size, max_blocks_per_seq, num_blocks, dtype, scale, out, partition_tokens,
+                          workspace, workspace_bytes, stream);
 }
 
 int paged_attn_decode_gqa_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
