@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline time budget")
+    ap.add_argument("--q-len", type=int, default=1,
+                    help="query tokens per sequence (>1: verify / chunked-prefill step through "
+                         "paged_attn_multi_query; the last q_len positions are appended each step)")
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="profiling aid: fewer sequences of the opt13b layer (a smaller case for ncu)")
     a = ap.parse_args()
@@ -294,14 +297,42 @@ def run_gpu(a, rank, world, local_rank):
         w = wl.make(a.workload, device=dev, B=a.block_size if a.workload in ("opt13b",) or
                     a.workload.startswith("gqa") else None)
     pt = w.partition_tokens if a.partition_tokens is None else a.partition_tokens
+    Lq = a.q_len
+    if Lq > 1:
+        # the step's Lq new tokens are the last Lq positions of each context
+        sl = np.full((w.S, Lq), -1, dtype=np.int64)
+        for s_ in range(w.S):
+            c = int(w.context_lens[s_])
+            for j in range(Lq):
+                pos = c - Lq + j
+                if pos >= 0:
+                    sl[s_, j] = int(w.block_tables[s_, pos // w.B]) * w.B + pos % w.B
+        w.slot_mapping = sl.reshape(-1)
+        gq = torch.Generator(device=dev)
+        gq.manual_seed(4242)
+        w.q = torch.randn((w.S, Lq, w.H, w.D), generator=gq, device=dev).to(w.q.dtype)
+        w.k_new = torch.randn((w.S * Lq, w.Hkv, w.D), generator=gq, device=dev).to(w.q.dtype)
+        w.v_new = torch.randn((w.S * Lq, w.Hkv, w.D), generator=gq, device=dev).to(w.q.dtype)
     bt = torch.from_numpy(w.block_tables).to(dev)
     ctx = torch.from_numpy(w.context_lens).to(dev)
     slots = torch.from_numpy(w.slot_mapping).to(dev)
     pairs = torch.from_numpy(w.cow_pairs.reshape(-1, 2)).to(dev)
-    out = torch.empty((w.S, w.H, w.D), dtype=torch.float32, device=dev)
-    ws = pkv.alloc_workspace(w.q, w.k_pool, bt, pt)
-    pt_used = pkv.gqa_partition_tokens(w.S, w.H, w.Hkv, w.D, w.B, w.max_blocks, pt)
+    out = torch.empty(tuple(w.q.shape), dtype=torch.float32, device=dev)
+    if Lq > 1:
+        nws = pkv.load().paged_attn_multi_query_workspace_size(w.S, Lq, w.H, w.Hkv, w.D, w.B, w.max_blocks, pt)
+        ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+        pt_used = pt if pt else pkv.gqa_partition_tokens(w.S, w.H, w.Hkv, w.D, w.B, w.max_blocks, 0)
+    else:
+        ws = pkv.alloc_workspace(w.q, w.k_pool, bt, pt)
+        pt_used = pkv.gqa_partition_tokens(w.S, w.H, w.Hkv, w.D, w.B, w.max_blocks, pt)
     split = pt_used < w.max_blocks * w.B
+
+    def attend(qt):
+        if Lq > 1:
+            return pkv.paged_attn_multi_query(qt, w.k_pool, w.v_pool, bt, ctx, w.scale, out=out,
+                                              partition_tokens=pt, workspace=ws)
+        return pkv.paged_attn_decode(qt, w.k_pool, w.v_pool, bt, ctx, w.scale, out=out, partition_tokens=pt,
+                                     workspace=ws)
     stream = torch.cuda.current_stream(dev)
     launches_per_step = (1 if len(w.cow_pairs) else 0) + 1 + 2 + (1 if split else 0)
 
@@ -311,8 +342,7 @@ def run_gpu(a, rank, world, local_rank):
         pkv.kv_cache_append(w.k_new, w.v_new, w.k_pool, w.v_pool, slots)
         if dec_events is not None:
             dec_events[0].record(stream)
-        pkv.paged_attn_decode(w.q, w.k_pool, w.v_pool, bt, ctx, w.scale, out=out, partition_tokens=pt,
-                              workspace=ws)
+        attend(w.q)
         if dec_events is not None:
             dec_events[1].record(stream)
 
@@ -371,8 +401,12 @@ def run_gpu(a, rank, world, local_rank):
         if len(w.cow_pairs):
             pkv.kv_block_copy(w.k_pool, w.v_pool, dpr)
         pkv.kv_cache_append(dk, dv, w.k_pool, w.v_pool, dsl)
-        pkv.paged_attn_decode(dq, w.k_pool, w.v_pool, dbt, dctx, w.scale, out=out, partition_tokens=pt,
-                              workspace=ws)
+        if Lq > 1:
+            pkv.paged_attn_multi_query(dq, w.k_pool, w.v_pool, dbt, dctx, w.scale, out=out, partition_tokens=pt,
+                                       workspace=ws)
+        else:
+            pkv.paged_attn_decode(dq, w.k_pool, w.v_pool, dbt, dctx, w.scale, out=out, partition_tokens=pt,
+                                  workspace=ws)
         out_h.copy_(out, non_blocking=True)
 
     for _ in range(a.warmup):
@@ -415,6 +449,7 @@ def run_gpu(a, rank, world, local_rank):
             "block_size": w.B,
             "context_tokens_per_step": int(w.context_lens.sum()), "kv_bytes_per_step": kv_bytes,
             "cow_pairs_per_step": int(len(w.cow_pairs)), "appended_tokens_per_step": int((w.slot_mapping >= 0).sum()),
+            "query_tokens_per_sequence": Lq,
             "partition_tokens": pt_used,
             "l2": f"no flush: K/V pool {w.k_pool.numel() * w.k_pool.element_size() * 2 / 1e9:.2f} GB "
                   f"= {w.k_pool.numel() * w.k_pool.element_size() * 2 / 126e6:.0f}x L2",
@@ -424,7 +459,8 @@ def run_gpu(a, rank, world, local_rank):
         "seq_per_s": round(w.S * world / (ms_step * 1e-3), 1),
         "ctx_tokens_per_s": round(int(w.context_lens.sum()) * world / (ms_step * 1e-3), 1),
         "roofline": {
-            "kernel": "paged_attn_decode call (plan + persistent decode + merge launches)",
+            "kernel": ("paged_attn_multi_query" if Lq > 1 else "paged_attn_decode") +
+                      " call (plan + persistent attention kernel + merge launches)",
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
