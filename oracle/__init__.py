@@ -13,7 +13,10 @@ checked against the pages by eye:
 * ``paged_attention``  gather a sequence's K/V through its block table into a
                        contiguous array, then softmax(scale * K q) V.
 * ``cache_ops``        per-token append into slots, copy-on-write block copy,
-                       and the plain gather used to check indexing.
+                       block swaps to and from host memory, and the plain
+                       gather used to check indexing.
+* ``block_manager``    the host bookkeeping: free list, reference counts,
+                       on-demand blocks, copy-on-write trigger, swap lists.
 
 Sources (cited by page title and section):
 
@@ -42,7 +45,8 @@ from .paged_attention import (
     paged_decode_selected,
     paged_multi_query,
 )
-from .cache_ops import kv_append, kv_block_copy, gather_kv
+from .cache_ops import kv_append, kv_block_copy, gather_kv, kv_swap_out, kv_swap_in
+from .block_manager import BlockManager, BlockManagerError
 
 __all__ = [
     "to_f64",
@@ -56,4 +60,8 @@ __all__ = [
     "kv_append",
     "kv_block_copy",
     "gather_kv",
+    "kv_swap_out",
+    "kv_swap_in",
+    "BlockManager",
+    "BlockManagerError",
 ]

@@ -81,3 +81,37 @@ def gather_kv(pool, table_row, ctx, block_size):
             raise IndexError("block table entry outside the pool")
         out[:, t, :] = pool[phys, :, t % block_size, :]
     return out
+
+
+def kv_swap_out(k_pool, v_pool, block_ids):
+    """Return ``(host_k, host_v, n_bad)`` with ``host[i] = pool[block_ids[i]]`` (all heads and slots).
+
+    Swapping a preempted sequence's blocks to host memory ("PagedAttention - Efficient
+    Memory Management for LLM Serving with vLLM", section "Method", scheduling).  An id
+    outside the pool leaves its host slot zero and is counted in ``n_bad``.
+    """
+    ids = np.asarray(block_ids).reshape(-1)
+    hk = np.zeros((len(ids),) + k_pool.shape[1:], dtype=k_pool.dtype)
+    hv = np.zeros((len(ids),) + v_pool.shape[1:], dtype=v_pool.dtype)
+    n_bad = 0
+    for i, b in enumerate(ids.tolist()):
+        if not (0 <= b < k_pool.shape[0]):
+            n_bad += 1
+            continue
+        hk[i] = k_pool[b]
+        hv[i] = v_pool[b]
+    return hk, hv, n_bad
+
+
+def kv_swap_in(k_pool, v_pool, host_k, host_v, block_ids):
+    """Return ``(k_pool', v_pool', n_bad)`` with ``pool'[block_ids[i]] = host[i]``."""
+    k = np.array(k_pool, copy=True)
+    v = np.array(v_pool, copy=True)
+    n_bad = 0
+    for i, b in enumerate(np.asarray(block_ids).reshape(-1).tolist()):
+        if not (0 <= b < k.shape[0]):
+            n_bad += 1
+            continue
+        k[b] = host_k[i]
+        v[b] = host_v[i]
+    return k, v, n_bad
