@@ -37,9 +37,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention effective KV GB/s and % of B200 HBM peak"
 FALLBACK_HBM_GBS = 6650.0
-WORKLOADS = ("opt13b", "llama7b", "cow", "longctx", "tiny", "gqa2", "gqa4", "gqa8", "gqa16")
+WORKLOADS = ("opt13b", "llama7b", "cow", "longctx", "tiny", "gqa2", "gqa4", "gqa8", "gqa16", "swap")
 DEFAULT_STEPS = {"opt13b": 500, "llama7b": 2000, "cow": 1000, "longctx": 500, "tiny": 200,
-                 "gqa2": 500, "gqa4": 500, "gqa8": 500, "gqa16": 500}
+                 "gqa2": 500, "gqa4": 500, "gqa8": 500, "gqa16": 500, "swap": 20}
 
 
 def parse():
@@ -528,6 +528,57 @@ def run_reference(a, rank, world):
     print(json.dumps(res), flush=True)
 
 
+def run_swap(a, rank, world, local_rank):
+    """Block-granular swap: every step moves 1024 random blocks of the batch-256
+    layer's pool (B=16: 160 KB of K and 160 KB of V each) to pinned host memory and
+    back into other free blocks.  Metric: bytes moved per direction per second."""
+    import torch
+    import paged_kv_cache_328_b200 as pkv
+    from paged_kv_cache_328_b200 import workloads as wl
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pkv.load()
+    w = wl.make_opt13b(B=a.block_size, device=dev)
+    n = 1024
+    rng = np.random.default_rng(11)
+    perm = rng.permutation(w.num_blocks)
+    out_ids = torch.from_numpy(perm[:n].astype(np.int64)).to(dev)
+    in_ids = torch.from_numpy(perm[n:2 * n].astype(np.int64)).to(dev)
+    shape = (n,) + tuple(w.k_pool.shape[1:])
+    hk = torch.empty(shape, dtype=w.k_pool.dtype).pin_memory()
+    hv = torch.empty(shape, dtype=w.k_pool.dtype).pin_memory()
+    st = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for _ in range(a.warmup):
+        pkv.kv_blocks_to_host(w.k_pool, w.v_pool, out_ids, hk, hv)
+        pkv.kv_blocks_from_host(hk, hv, w.k_pool, w.v_pool, in_ids)
+    torch.cuda.synchronize()
+    t_out = t_in = 0.0
+    for _ in range(a.steps):
+        ev[0].record(st)
+        pkv.kv_blocks_to_host(w.k_pool, w.v_pool, out_ids, hk, hv)
+        ev[1].record(st)
+        pkv.kv_blocks_from_host(hk, hv, w.k_pool, w.v_pool, in_ids)
+        ev[2].record(st)
+        torch.cuda.synchronize()
+        t_out += ev[0].elapsed_time(ev[1])
+        t_in += ev[1].elapsed_time(ev[2])
+    code, reason = pkv.get_device_error(dev)
+    if code != 0:
+        raise RuntimeError(f"device error word: {code} reason {reason}")
+    moved = 2 * n * hk[0].numel() * hk.element_size()
+    res = {"metric": "KV block swap GB/s (device <-> pinned host, one kernel per direction)",
+           "value": round(moved / ((t_out + t_in) / 2 / a.steps * 1e-3) / 1e9, 2), "unit": "GB/s",
+           "to_host_gbs": round(moved / (t_out / a.steps * 1e-3) / 1e9, 2),
+           "from_host_gbs": round(moved / (t_in / a.steps * 1e-3) / 1e9, 2),
+           "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+           "ms_per_step": round((t_out + t_in) / a.steps, 4), "higher_is_better": True, "dtype": w.dtype,
+           "data": "synthetic", "config": {"workload": "swap", "blocks_per_direction": n,
+                                           "bytes_per_direction": moved, "block_size": w.B}}
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
 def main():
     a = parse()
     rank, world, local_rank = dist_env()
@@ -535,6 +586,9 @@ def main():
         print(f"warning: --gpus {a.gpus} but WORLD_SIZE {world}", file=sys.stderr)
     if a.impl == "reference":
         run_reference(a, rank, world)
+        return
+    if a.workload == "swap":
+        run_swap(a, rank, world, local_rank)
         return
     run_gpu(a, rank, world, local_rank)
 

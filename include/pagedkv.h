@@ -66,7 +66,9 @@ enum {
   PKV_ECUDA = -5,         /* a CUDA runtime call or a kernel launch failed */
   PKV_EWORKSPACE = -6,    /* workspace smaller than paged_attn_decode_workspace_size() */
   PKV_EDEVICE = -7,       /* a kernel flagged bad device data (see pkv_get_device_error) */
-  PKV_ETIMEOUT = -8       /* a kernel's bounded wait ran out (see pkv_get_device_error) */
+  PKV_ETIMEOUT = -8,      /* a kernel's bounded wait ran out (see pkv_get_device_error) */
+  PKV_ENOMEM = -9,        /* block manager: not enough free blocks (nothing was changed) */
+  PKV_ESEQ = -10          /* block manager: unknown sequence, sequence exists, or repeated in a batch */
 };
 
 /* Reasons stored in the device error word (the `reason` of pkv_get_device_error). */
@@ -254,6 +256,77 @@ int kv_block_copy(void* k_cache, void* v_cache, const int64_t* src_dst_pairs,
 int paged_kv_gather(const void* cache, const int32_t* block_table_row, int context_len,
                     int num_heads, int head_dim, int block_size, int num_blocks,
                     pkv_dtype dtype, void* out, void* stream);
+
+/*
+ * kv_blocks_to_host / kv_blocks_from_host - block-granular swap of the cache to and
+ * from pinned host memory (a preempted sequence's blocks move to host RAM and back:
+ * "PagedAttention - Efficient Memory Management for LLM Serving with vLLM", section
+ * "Method", scheduling).
+ *
+ *   to host:   host_k[i] = k_cache[block_ids[i]] and host_v[i] = v_cache[block_ids[i]]
+ *   from host: k_cache[block_ids[i]] = host_k[i] and v_cache[block_ids[i]] = host_v[i]
+ * for i < num_blocks_moved, every head and slot, bit for bit, in one kernel launch
+ * that reads or writes host memory directly over the host link.
+ *
+ *   block_ids     int64 [num_blocks_moved], device memory.
+ *   host_k,
+ *   host_v        pinned (page-locked) host memory, [num_blocks_moved][num_heads]
+ *                 [block_size][head_dim] each, 16-byte aligned; memory that is not
+ *                 page-locked is rejected with PKV_EINVAL.
+ * An id outside [0, num_blocks) is skipped and flagged (PKV_DEV_COPY_PAIR).  The
+ * host buffers must not be touched by the host until the stream has passed the call.
+ */
+int kv_blocks_to_host(const void* k_cache, const void* v_cache, const int64_t* block_ids,
+                      int num_blocks_moved, void* host_k, void* host_v, int num_heads,
+                      int head_dim, int block_size, int num_blocks, pkv_dtype dtype, void* stream);
+int kv_blocks_from_host(const void* host_k, const void* host_v, void* k_cache, void* v_cache,
+                        const int64_t* block_ids, int num_blocks_moved, int num_heads,
+                        int head_dim, int block_size, int num_blocks, pkv_dtype dtype,
+                        void* stream);
+
+/*
+ * Block manager: host bookkeeping of the physical block pool (pure host code, no
+ * CUDA call).  Blocks come from the front of a FIFO free list with reference count
+ * 1 and return to its back when the count reaches 0 ("vLLM PagedAttention and
+ * continuous batching", section 4); a sequence of n tokens holds ceil(n / B)
+ * blocks, taken on demand ("LLM Inference 8 - PagedAttention", section
+ * "PagedAttention의 동작 방식"); forked sequences share blocks, and an append into a
+ * shared last block copies it first (copy-on-write, the paper digest's flowchart).
+ * Calls on one manager are serialised by an internal mutex.  Sequence ids are any
+ * int64 values.  Errors: PKV_EINVAL (bad argument), PKV_ESEQ, PKV_ENOMEM; a failed
+ * call changes nothing.
+ */
+typedef struct pkv_block_manager pkv_block_manager;
+
+/* free_order: NULL for 0, 1, ..., num_blocks - 1, else a permutation of them. NULL on bad arguments. */
+pkv_block_manager* pkv_bm_create(int num_blocks, int block_size, const int32_t* free_order);
+void pkv_bm_destroy(pkv_block_manager* bm);
+/* A new sequence holding num_tokens tokens (a prompt): takes ceil(num_tokens / B) blocks. */
+int pkv_bm_add_sequence(pkv_block_manager* bm, int64_t seq, int num_tokens);
+/* child shares every block of parent (reference counts + 1). */
+int pkv_bm_fork(pkv_block_manager* bm, int64_t parent, int64_t child);
+/*
+ * One new token for each of the n distinct sequences: slots[i] receives the slot of
+ * seqs[i]'s new token (for kv_cache_append); each copy-on-write appends its
+ * (src, dst) pair to cow_pairs (capacity 2 * n entries; for kv_block_copy) and
+ * *num_pairs counts them.
+ */
+int pkv_bm_append_tokens(pkv_block_manager* bm, const int64_t* seqs, int n, int64_t* slots,
+                         int64_t* cow_pairs, int* num_pairs);
+/* Releases the sequence's blocks (or forgets a swapped-out sequence). */
+int pkv_bm_free_sequence(pkv_block_manager* bm, int64_t seq);
+/* Copies the block table (padded with -1 to max_blocks) and the token count; returns the block count. */
+int pkv_bm_block_table(pkv_block_manager* bm, int64_t seq, int32_t* row, int max_blocks,
+                       int64_t* num_tokens);
+/* Block tables [n][max_blocks] and context lengths [n] of n sequences: the decode step's inputs. */
+int pkv_bm_fill_tables(pkv_block_manager* bm, const int64_t* seqs, int n, int32_t* block_tables,
+                       int max_blocks, int32_t* context_lens);
+int pkv_bm_num_free(pkv_block_manager* bm);
+int pkv_bm_ref_count(pkv_block_manager* bm, int block);
+/* Lists the sequence's blocks in logical order (copy them with kv_blocks_to_host), then releases them. */
+int pkv_bm_swap_out(pkv_block_manager* bm, int64_t seq, int64_t* blocks, int max_blocks, int* n_blocks);
+/* Takes fresh blocks for a swapped-out sequence: host slot i goes to blocks[i] (kv_blocks_from_host). */
+int pkv_bm_swap_in(pkv_block_manager* bm, int64_t seq, int64_t* blocks, int max_blocks, int* n_blocks);
 
 /*
  * pkv_get_device_error - synchronise `stream`, read and clear the device error

@@ -8,7 +8,9 @@ The hot path is a C-ABI shared library, ``libpagedkv.so`` (declared in
                          log-sum-exp;
 * ``kv_cache_append``    per-token K/V append into slots;
 * ``kv_block_copy``      copy-on-write block copies;
-* ``paged_kv_gather``    contiguous copy of one sequence (indexing checks).
+* ``paged_kv_gather``    contiguous copy of one sequence (indexing checks);
+* ``kv_blocks_to_host`` / ``kv_blocks_from_host``  block-granular swaps;
+* ``BlockManager``       the native host-side block bookkeeping.
 
 This package is the thin Python binding (argument marshalling only) plus the
 seeded synthetic input generator in ``workloads``.  Nothing here computes on the
@@ -16,6 +18,7 @@ CPU: without the built library every call raises.
 """
 
 from ._lib import (  # noqa: F401
+    BlockManager,
     PagedKVError,
     abi_version,
     alloc_workspace,
@@ -23,6 +26,8 @@ from ._lib import (  # noqa: F401
     gqa_partition_tokens,
     gqa_workspace_size,
     kv_block_copy,
+    kv_blocks_from_host,
+    kv_blocks_to_host,
     kv_cache_append,
     load,
     paged_attn_decode,

@@ -19,7 +19,8 @@ DTYPE_CODE = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PK
 
 ERRORS = {
     0: "PKV_OK", -1: "PKV_EINVAL", -2: "PKV_EDTYPE", -3: "PKV_EALIGN", -4: "PKV_EUNSUPPORTED",
-    -5: "PKV_ECUDA", -6: "PKV_EWORKSPACE", -7: "PKV_EDEVICE", -8: "PKV_ETIMEOUT",
+    -5: "PKV_ECUDA", -6: "PKV_EWORKSPACE", -7: "PKV_EDEVICE", -8: "PKV_ETIMEOUT", -9: "PKV_ENOMEM",
+    -10: "PKV_ESEQ",
 }
 DEVICE_REASONS = {0: "ok", 1: "block id", 2: "context length", 3: "slot", 4: "copy pair", 5: "wait timeout"}
 
@@ -45,6 +46,22 @@ SIGNATURES = {
     "paged_attn_multi_query": (_c_int, [_c_void_p] * 5 + [_c_int] * 9 + [_c_float, _c_void_p, _c_int, _c_void_p,
                                                                      _c_size_t, _c_void_p]),
     "paged_attn_multi_query_workspace_size": (_c_size_t, [_c_int] * 8),
+    "kv_blocks_to_host": (_c_int, [_c_void_p] * 3 + [_c_int] + [_c_void_p] * 2 + [_c_int] * 5 + [_c_void_p]),
+    "kv_blocks_from_host": (_c_int, [_c_void_p] * 5 + [_c_int] * 6 + [_c_void_p]),
+    "pkv_bm_create": (_c_void_p, [_c_int, _c_int, _c_void_p]),
+    "pkv_bm_destroy": (None, [_c_void_p]),
+    "pkv_bm_add_sequence": (_c_int, [_c_void_p, ctypes.c_int64, _c_int]),
+    "pkv_bm_fork": (_c_int, [_c_void_p, ctypes.c_int64, ctypes.c_int64]),
+    "pkv_bm_append_tokens": (_c_int, [_c_void_p, _c_void_p, _c_int, _c_void_p, _c_void_p,
+                                      ctypes.POINTER(_c_int)]),
+    "pkv_bm_free_sequence": (_c_int, [_c_void_p, ctypes.c_int64]),
+    "pkv_bm_block_table": (_c_int, [_c_void_p, ctypes.c_int64, _c_void_p, _c_int,
+                                    ctypes.POINTER(ctypes.c_int64)]),
+    "pkv_bm_fill_tables": (_c_int, [_c_void_p, _c_void_p, _c_int, _c_void_p, _c_int, _c_void_p]),
+    "pkv_bm_num_free": (_c_int, [_c_void_p]),
+    "pkv_bm_ref_count": (_c_int, [_c_void_p, _c_int]),
+    "pkv_bm_swap_out": (_c_int, [_c_void_p, ctypes.c_int64, _c_void_p, _c_int, ctypes.POINTER(_c_int)]),
+    "pkv_bm_swap_in": (_c_int, [_c_void_p, ctypes.c_int64, _c_void_p, _c_int, ctypes.POINTER(_c_int)]),
     "paged_attn_decode_noalloc": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                            _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                            _c_float, _c_void_p, _c_int, _c_void_p]),
@@ -318,3 +335,129 @@ def paged_attn_multi_query(q, k_cache, v_cache, block_tables, context_lens, scal
         rc = lib.paged_attn_multi_query(*args, _stream(q.device, stream))
     _check(rc, "paged_attn_multi_query")
     return out
+
+
+def _host_pinned(t, name):
+    if not isinstance(t, torch.Tensor) or t.device.type != "cpu" or not t.is_pinned() or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous pinned (page-locked) CPU tensor")
+    return t.data_ptr()
+
+
+def kv_blocks_to_host(k_cache, v_cache, block_ids, host_k, host_v, stream=None):
+    """host_k[i] = k_cache[block_ids[i]] (and V) into pinned host tensors [n, H, B, D]."""
+    lib = load()
+    NB, H, B, D = k_cache.shape
+    n = block_ids.numel()
+    if tuple(host_k.shape) != (n, H, B, D) or host_v.shape != host_k.shape or host_k.dtype != k_cache.dtype:
+        raise ValueError("host buffers must be [n, H, B, D] in the cache dtype")
+    args = (_cuda(k_cache, "k_cache", DTYPE_CODE), _cuda(v_cache, "v_cache", DTYPE_CODE),
+            _cuda(block_ids, "block_ids", (torch.int64,)), n, _host_pinned(host_k, "host_k"),
+            _host_pinned(host_v, "host_v"), H, D, B, NB, DTYPE_CODE[k_cache.dtype])
+    with torch.cuda.device(k_cache.device):
+        rc = lib.kv_blocks_to_host(*args, _stream(k_cache.device, stream))
+    _check(rc, "kv_blocks_to_host")
+
+
+def kv_blocks_from_host(host_k, host_v, k_cache, v_cache, block_ids, stream=None):
+    """k_cache[block_ids[i]] = host_k[i] (and V) from pinned host tensors [n, H, B, D]."""
+    lib = load()
+    NB, H, B, D = k_cache.shape
+    n = block_ids.numel()
+    if tuple(host_k.shape) != (n, H, B, D) or host_v.shape != host_k.shape or host_k.dtype != k_cache.dtype:
+        raise ValueError("host buffers must be [n, H, B, D] in the cache dtype")
+    args = (_host_pinned(host_k, "host_k"), _host_pinned(host_v, "host_v"),
+            _cuda(k_cache, "k_cache", DTYPE_CODE), _cuda(v_cache, "v_cache", DTYPE_CODE),
+            _cuda(block_ids, "block_ids", (torch.int64,)), n, H, D, B, NB, DTYPE_CODE[k_cache.dtype])
+    with torch.cuda.device(k_cache.device):
+        rc = lib.kv_blocks_from_host(*args, _stream(k_cache.device, stream))
+    _check(rc, "kv_blocks_from_host")
+
+
+class BlockManager:
+    """The library's native block manager (host code; no GPU needed).
+
+    Free list, reference counts and per-sequence block tables of one physical
+    block pool; see include/pagedkv.h.  Methods raise PagedKVError on failure
+    (a failed call changes nothing).
+    """
+
+    def __init__(self, num_blocks, block_size, free_order=None):
+        self._lib = load()
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+        arr = None
+        if free_order is not None:
+            arr = (ctypes.c_int32 * num_blocks)(*[int(b) for b in free_order])
+        self._h = self._lib.pkv_bm_create(self.num_blocks, self.block_size, arr)
+        if not self._h:
+            raise PagedKVError(-1, "pkv_bm_create")
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.pkv_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    def _rc(self, rc, where):
+        if rc < 0:
+            raise PagedKVError(rc, where)
+        return rc
+
+    def add_sequence(self, seq, num_tokens):
+        self._rc(self._lib.pkv_bm_add_sequence(self._h, int(seq), int(num_tokens)), "pkv_bm_add_sequence")
+
+    def fork(self, parent, child):
+        self._rc(self._lib.pkv_bm_fork(self._h, int(parent), int(child)), "pkv_bm_fork")
+
+    def append_tokens(self, seqs):
+        """One token for each sequence: (slots, [(src, dst), ...] copy-on-write pairs)."""
+        n = len(seqs)
+        seq_arr = (ctypes.c_int64 * max(1, n))(*[int(x) for x in seqs])
+        slots = (ctypes.c_int64 * max(1, n))()
+        pairs = (ctypes.c_int64 * max(2, 2 * n))()
+        npairs = ctypes.c_int(0)
+        self._rc(self._lib.pkv_bm_append_tokens(self._h, seq_arr, n, slots, pairs, ctypes.byref(npairs)),
+                 "pkv_bm_append_tokens")
+        return list(slots[:n]), [(pairs[2 * i], pairs[2 * i + 1]) for i in range(npairs.value)]
+
+    def free_sequence(self, seq):
+        self._rc(self._lib.pkv_bm_free_sequence(self._h, int(seq)), "pkv_bm_free_sequence")
+
+    def block_table(self, seq, max_blocks=None):
+        cap = self.num_blocks if max_blocks is None else int(max_blocks)
+        row = (ctypes.c_int32 * max(1, cap))()
+        tokens = ctypes.c_int64(0)
+        n = self._rc(self._lib.pkv_bm_block_table(self._h, int(seq), row, cap, ctypes.byref(tokens)),
+                     "pkv_bm_block_table")
+        return list(row[:n]), tokens.value
+
+    def fill_tables(self, seqs, max_blocks):
+        """Block tables int32 [n, max_blocks] (-1 padded) and context lengths int32 [n] as CPU tensors."""
+        n = len(seqs)
+        seq_arr = (ctypes.c_int64 * max(1, n))(*[int(x) for x in seqs])
+        tables = torch.empty((n, max_blocks), dtype=torch.int32)
+        lens = torch.empty((n,), dtype=torch.int32)
+        self._rc(self._lib.pkv_bm_fill_tables(self._h, seq_arr, n, tables.data_ptr(), int(max_blocks),
+                                              lens.data_ptr()), "pkv_bm_fill_tables")
+        return tables, lens
+
+    def num_free(self):
+        return self._rc(self._lib.pkv_bm_num_free(self._h), "pkv_bm_num_free")
+
+    def ref_count(self, block):
+        return self._rc(self._lib.pkv_bm_ref_count(self._h, int(block)), "pkv_bm_ref_count")
+
+    def swap_out(self, seq):
+        blocks = (ctypes.c_int64 * max(1, self.num_blocks))()
+        n = ctypes.c_int(0)
+        self._rc(self._lib.pkv_bm_swap_out(self._h, int(seq), blocks, self.num_blocks, ctypes.byref(n)),
+                 "pkv_bm_swap_out")
+        return list(blocks[:n.value])
+
+    def swap_in(self, seq):
+        blocks = (ctypes.c_int64 * max(1, self.num_blocks))()
+        n = ctypes.c_int(0)
+        self._rc(self._lib.pkv_bm_swap_in(self._h, int(seq), blocks, self.num_blocks, ctypes.byref(n)),
+                 "pkv_bm_swap_in")
+        return list(blocks[:n.value])

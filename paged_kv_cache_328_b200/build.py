@@ -2,9 +2,10 @@
 
     python -m paged_kv_cache_328_b200.build [--force] [--verbose]
 
-The library is one translation unit (csrc/pagedkv.cu includes the kernel
-headers) compiled for ``sm_100a`` only; the CUDA runtime is linked statically, so
-the .so needs nothing but the driver at run time.
+The library is csrc/pagedkv.cu (the C ABI; it includes the kernel headers)
+compiled for ``sm_100a`` only, plus the host-only block manager
+(csrc/block_manager.cpp); the CUDA runtime is linked statically, so the .so
+needs nothing but the driver at run time.
 """
 
 import argparse
@@ -19,7 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpagedkv.so")
-MAIN = os.path.join(CSRC, "pagedkv.cu")
+MAIN = [os.path.join(CSRC, "pagedkv.cu"), os.path.join(CSRC, "block_manager.cpp")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-shared", "--expt-relaxed-constexpr"]
@@ -36,7 +37,7 @@ def nvcc():
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
-                  glob.glob(os.path.join(INCLUDE, "*.h")))
+                  glob.glob(os.path.join(CSRC, "*.cpp")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
 def up_to_date():
@@ -50,7 +51,7 @@ def build(force=False, verbose=False):
     """Compile the library if a source is newer than it (or ``force``); return its path."""
     if not force and up_to_date():
         return LIB
-    cmd = [nvcc()] + ARCH + FLAGS + ["-I", INCLUDE, "-o", LIB + ".tmp", MAIN]
+    cmd = [nvcc()] + ARCH + FLAGS + ["-I", INCLUDE, "-o", LIB + ".tmp"] + MAIN
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)

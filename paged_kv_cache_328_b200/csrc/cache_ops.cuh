@@ -66,6 +66,36 @@ __global__ void __launch_bounds__(kCopyThreads)
   }
 }
 
+// kv_blocks_to_host / kv_blocks_from_host: grid = (chunks per block, blocks, 2 for K|V).
+// Slot i of the host buffers is block ids[i] of the pool; the host side is pinned
+// memory reached through its device address (loads or stores cross the host link).
+__global__ void __launch_bounds__(kCopyThreads)
+    kv_swap_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache, uint4* __restrict__ host_k,
+                   uint4* __restrict__ host_v, const int64_t* __restrict__ ids, long long block_vecs, int num_blocks,
+                   int to_host) {
+  const long long b = ids[blockIdx.y];
+  if (b < 0 || b >= num_blocks) {
+    if (blockIdx.x == 0 && blockIdx.z == 0 && threadIdx.x == 0) flag_error(PKV_DEV_COPY_PAIR);
+    return;
+  }
+  uint4* pool = (blockIdx.z ? v_cache : k_cache) + (size_t)b * block_vecs;
+  uint4* host = (blockIdx.z ? host_v : host_k) + (size_t)blockIdx.y * block_vecs;
+  const uint4* from = to_host ? pool : host;
+  uint4* to = to_host ? host : pool;
+  const long long base = (long long)blockIdx.x * (kCopyThreads * kCopyVecs) + threadIdx.x;
+  uint4 buf[kCopyVecs];
+#pragma unroll
+  for (int j = 0; j < kCopyVecs; ++j) {
+    const long long idx = base + (long long)j * kCopyThreads;
+    if (idx < block_vecs) buf[j] = from[idx];
+  }
+#pragma unroll
+  for (int j = 0; j < kCopyVecs; ++j) {
+    const long long idx = base + (long long)j * kCopyThreads;
+    if (idx < block_vecs) to[idx] = buf[j];
+  }
+}
+
 // paged_kv_gather: out[h][t][:] = cache[table[t / B]][h][t % B][:].  Rows are
 // addressed with pool_row, the helper the decode kernel's producer uses.
 __global__ void __launch_bounds__(256)

@@ -612,6 +612,66 @@ int kv_block_copy(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, in
   return PKV_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Device address of pinned host memory, or nullptr if `p` is not page-locked host memory.
+void* pinned_device_address(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || a.devicePointer == nullptr) return nullptr;
+  return a.devicePointer;
+}
+
+int swap_impl(void* k_cache, void* v_cache, void* host_k, void* host_v, const int64_t* block_ids, int n,
+              int num_heads, int head_dim, int block_size, int num_blocks, pkv_dtype dtype, void* stream,
+              int to_host) {
+  const int e = elem_bytes(dtype);
+  if (e == 0) return PKV_EDTYPE;
+  if (n < 0 || num_heads <= 0 || num_blocks <= 0) return PKV_EINVAL;
+  if (!head_dim_ok(head_dim) || !block_size_ok(block_size)) return PKV_EUNSUPPORTED;
+  if (n == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !host_k || !host_v || !block_ids) return PKV_EINVAL;
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(host_k, 16) || !aligned(host_v, 16) ||
+      !aligned(block_ids, 8))
+    return PKV_EALIGN;
+  if (n > 65535) return PKV_EINVAL;
+  void* dk = pinned_device_address(host_k);
+  void* dv = pinned_device_address(host_v);
+  if (!dk || !dv) return PKV_EINVAL;
+  const long long block_vecs = (long long)num_heads * block_size * head_dim * e / 16;
+  const long long per_cta = (long long)pkv::kCopyThreads * pkv::kCopyVecs;
+  const long long chunks = (block_vecs + per_cta - 1) / per_cta;
+  if (chunks > INT_MAX) return PKV_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  pkv::kv_swap_kernel<<<dim3((unsigned)chunks, (unsigned)n, 2), pkv::kCopyThreads, 0, st>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<uint4*>(dk), static_cast<uint4*>(dv),
+      block_ids, block_vecs, num_blocks, to_host);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kv_blocks_to_host(const void* k_cache, const void* v_cache, const int64_t* block_ids, int num_blocks_moved,
+                      void* host_k, void* host_v, int num_heads, int head_dim, int block_size, int num_blocks,
+                      pkv_dtype dtype, void* stream) {
+  return swap_impl(const_cast<void*>(k_cache), const_cast<void*>(v_cache), host_k, host_v, block_ids,
+                   num_blocks_moved, num_heads, head_dim, block_size, num_blocks, dtype, stream, 1);
+}
+
+int kv_blocks_from_host(const void* host_k, const void* host_v, void* k_cache, void* v_cache, const int64_t* block_ids,
+                        int num_blocks_moved, int num_heads, int head_dim, int block_size, int num_blocks,
+                        pkv_dtype dtype, void* stream) {
+  return swap_impl(k_cache, v_cache, const_cast<void*>(host_k), const_cast<void*>(host_v), block_ids,
+                   num_blocks_moved, num_heads, head_dim, block_size, num_blocks, dtype, stream, 0);
+}
+
 int paged_kv_gather(const void* cache, const int32_t* block_table_row, int context_len, int num_heads, int head_dim,
                     int block_size, int num_blocks, pkv_dtype dtype, void* out, void* stream) {
   const int e = elem_bytes(dtype);
@@ -660,6 +720,8 @@ const char* pkv_strerror(int code) {
     case PKV_EWORKSPACE: return "workspace smaller than paged_attn_decode_workspace_size()";
     case PKV_EDEVICE: return "a kernel flagged bad device data (block id, context length, slot or copy pair)";
     case PKV_ETIMEOUT: return "a kernel's bounded shared-memory wait ran out";
+    case PKV_ENOMEM: return "block manager: not enough free blocks (nothing was changed)";
+    case PKV_ESEQ: return "block manager: unknown sequence, sequence already exists, or repeated in a batch";
   }
   return "unknown error code";
 }
