@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", choices=WORKLOADS, default="opt13b")
     ap.add_argument("--block-size", type=int, default=16)
+    ap.add_argument("--tune", action="store_true",
+                    help="choose the partition size by timing the candidates on the workload before warm-up")
     ap.add_argument("--partition-tokens", type=int, default=None,
                     help="split-context partition size (default: the workload's, else the library's choice)")
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
@@ -318,11 +320,15 @@ def run_gpu(a, rank, world, local_rank):
     slots = torch.from_numpy(w.slot_mapping).to(dev)
     pairs = torch.from_numpy(w.cow_pairs.reshape(-1, 2)).to(dev)
     out = torch.empty(tuple(w.q.shape), dtype=torch.float32, device=dev)
+    tuned = None
     if Lq > 1:
         nws = pkv.load().paged_attn_multi_query_workspace_size(w.S, Lq, w.H, w.Hkv, w.D, w.B, w.max_blocks, pt)
         ws = torch.empty(nws, dtype=torch.uint8, device=dev)
         pt_used = pt if pt else pkv.gqa_partition_tokens(w.S, w.H, w.Hkv, w.D, w.B, w.max_blocks, 0)
     else:
+        if a.tune:
+            pt, times = pkv.tune_partition_tokens(w.q, w.k_pool, w.v_pool, bt, ctx, w.scale, reps=5, out=out)
+            tuned = {str(k): round(v, 5) for k, v in times.items()}
         ws = pkv.alloc_workspace(w.q, w.k_pool, bt, pt)
         pt_used = pkv.gqa_partition_tokens(w.S, w.H, w.Hkv, w.D, w.B, w.max_blocks, pt)
     split = pt_used < w.max_blocks * w.B
@@ -514,6 +520,8 @@ def run_gpu(a, rank, world, local_rank):
     if w.name == "cow":
         result["config"]["cow_memory_saving"] = round(w.info["cow_saving"], 4)
     result["config"]["last_block_waste"] = round(wl.last_block_waste(w), 4)
+    if tuned is not None:
+        result["config"]["tuned_ms_per_call"] = tuned
 
     if pool is not None:
         nbytes, tokens, wall, passes = time_oracle(pool, sample, a.cpu_seconds)

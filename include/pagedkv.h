@@ -178,6 +178,37 @@ int paged_attn_decode_gqa_partition_tokens(int num_seqs, int num_heads, int num_
                                            int max_blocks_per_seq, int partition_tokens);
 
 /*
+ * paged_attn_decode_tune - choose the split-context partition size for these inputs
+ * by measurement (the digest's discussion asks whether block size should be tuned per
+ * model and workload rather than hard-coded; the partition size is the part that can
+ * be changed per call).
+ *
+ * Runs paged_attn_decode_gqa on the given inputs for each candidate partition size
+ * (no split, then 4096, 2048, ... 64 tokens that are multiples of block_size and
+ * shorter than the longest possible context): one untimed call and `reps` timed
+ * calls each, timed with CUDA events on `stream`.  Synchronises the stream.  Returns
+ * the fastest partition size (> 0) or a negative PKV_E* code; `out` ends up holding
+ * the decode result for the chosen size.  times_ms / candidates (may be NULL, up to
+ * max_candidates entries) receive the mean time per call and the candidate sizes;
+ * *num_candidates (may be NULL) the number of candidates (at most 8).
+ *
+ *   workspace     at least paged_attn_decode_tune_workspace_size() bytes (required).
+ *   Other arguments as in paged_attn_decode_gqa.
+ */
+int paged_attn_decode_tune(const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens,
+                           int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                           int block_size, int max_blocks_per_seq, int num_blocks,
+                           pkv_dtype dtype, float scale, float* out, void* workspace,
+                           size_t workspace_bytes, int reps, float* times_ms, int* candidates,
+                           int max_candidates, int* num_candidates, void* stream);
+
+/* Workspace bytes paged_attn_decode_tune needs (the largest over its candidates). */
+size_t paged_attn_decode_tune_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                             int head_dim, int block_size,
+                                             int max_blocks_per_seq);
+
+/*
  * paged_attn_multi_query - several query tokens per sequence over its paged context.
  *
  * For a prefill chunk appended to a cached prefix, or draft tokens checked in one

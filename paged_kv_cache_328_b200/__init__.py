@@ -35,5 +35,6 @@ from ._lib import (  # noqa: F401
     paged_kv_gather,
     partition_tokens,
     strerror,
+    tune_partition_tokens,
     workspace_size,
 )

@@ -46,6 +46,10 @@ SIGNATURES = {
     "paged_attn_multi_query": (_c_int, [_c_void_p] * 5 + [_c_int] * 9 + [_c_float, _c_void_p, _c_int, _c_void_p,
                                                                      _c_size_t, _c_void_p]),
     "paged_attn_multi_query_workspace_size": (_c_size_t, [_c_int] * 8),
+    "paged_attn_decode_tune": (_c_int, [_c_void_p] * 5 + [_c_int] * 8 + [_c_float, _c_void_p, _c_void_p,
+                                                                     _c_size_t, _c_int, _c_void_p, _c_void_p,
+                                                                     _c_int, ctypes.POINTER(_c_int), _c_void_p]),
+    "paged_attn_decode_tune_workspace_size": (_c_size_t, [_c_int] * 6),
     "kv_blocks_to_host": (_c_int, [_c_void_p] * 3 + [_c_int] + [_c_void_p] * 2 + [_c_int] * 5 + [_c_void_p]),
     "kv_blocks_from_host": (_c_int, [_c_void_p] * 5 + [_c_int] * 6 + [_c_void_p]),
     "pkv_bm_create": (_c_void_p, [_c_int, _c_int, _c_void_p]),
@@ -461,3 +465,31 @@ class BlockManager:
         self._rc(self._lib.pkv_bm_swap_in(self._h, int(seq), blocks, self.num_blocks, ctypes.byref(n)),
                  "pkv_bm_swap_in")
         return list(blocks[:n.value])
+
+
+def tune_partition_tokens(q, k_cache, v_cache, block_tables, context_lens, scale, reps=5, out=None, stream=None):
+    """Time the candidate partition sizes on these inputs; returns (best, {size: ms per call})."""
+    lib = load()
+    S, H, D = q.shape
+    NB, Hkv, B, Dc = k_cache.shape
+    if Dc != D or H % Hkv:
+        raise ValueError("q [S,H,D] and caches [NB,Hkv,B,D] disagree")
+    MB = block_tables.shape[1]
+    n = lib.paged_attn_decode_tune_workspace_size(S, H, Hkv, D, B, MB)
+    if n == ctypes.c_size_t(-1).value:
+        raise PagedKVError(-1, "paged_attn_decode_tune_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((S, H, D), dtype=torch.float32, device=q.device)
+    times = (ctypes.c_float * 8)()
+    cands = (ctypes.c_int * 8)()
+    nc = ctypes.c_int(0)
+    args = (_cuda(q, "q", DTYPE_CODE), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+            _cuda(block_tables, "block_tables", (torch.int32,)), _cuda(context_lens, "context_lens", (torch.int32,)),
+            S, H, Hkv, D, B, MB, NB, DTYPE_CODE[k_cache.dtype], float(scale), _cuda(out, "out", (torch.float32,)),
+            ws.data_ptr(), n, int(reps), times, cands, 8, ctypes.byref(nc))
+    with torch.cuda.device(q.device):
+        rc = lib.paged_attn_decode_tune(*args, _stream(q.device, stream))
+    if rc < 0:
+        raise PagedKVError(rc, "paged_attn_decode_tune")
+    return rc, {cands[i]: times[i] for i in range(nc.value)}

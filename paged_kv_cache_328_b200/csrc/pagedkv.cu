@@ -545,6 +545,87 @@ int paged_attn_multi_query(const void* q, const void* k_cache, const void* v_cac
                           workspace, workspace_bytes, stream);
 }
 
+int paged_attn_decode_tune(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                           const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                           int block_size, int max_blocks_per_seq, int num_blocks, pkv_dtype dtype, float scale,
+                           float* out, void* workspace, size_t workspace_bytes, int reps, float* times_ms,
+                           int* candidates, int max_candidates, int* num_candidates, void* stream) {
+  if (reps <= 0 || reps > 1000 || !workspace || max_candidates < 0) return PKV_EINVAL;
+  // candidates: no split, then 4096 ... 64 tokens that split the maximum context
+  const long long max_ctx = (long long)max_blocks_per_seq * block_size;
+  if (max_ctx <= 0 || max_ctx > INT_MAX / 2) return PKV_EINVAL;
+  int cand[8];
+  int nc = 0;
+  cand[nc++] = (int)max_ctx;
+  for (int pt = 4096; pt >= 64; pt /= 2)
+    if (pt % block_size == 0 && pt < max_ctx && nc < 8) cand[nc++] = pt;
+  for (int i = 0; i < nc; ++i) {
+    const size_t need = paged_attn_decode_gqa_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                                             max_blocks_per_seq, cand[i]);
+    if (need == (size_t)-1) return PKV_EINVAL;
+    if (need > workspace_bytes) return PKV_EWORKSPACE;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaEvent_t e0, e1;
+  if (cudaEventCreate(&e0) != cudaSuccess) return PKV_ECUDA;
+  if (cudaEventCreate(&e1) != cudaSuccess) {
+    cudaEventDestroy(e0);
+    return PKV_ECUDA;
+  }
+  int best = -1;
+  float best_ms = 0.f;
+  int rc = PKV_OK;
+  for (int i = 0; i < nc && rc == PKV_OK; ++i) {
+    // one untimed call, then `reps` timed back-to-back calls
+    for (int r = 0; r <= reps && rc == PKV_OK; ++r) {
+      if (r == 1 && cudaEventRecord(e0, st) != cudaSuccess) rc = PKV_ECUDA;
+      if (rc == PKV_OK)
+        rc = decode_impl(q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads, num_kv_heads,
+                         head_dim, block_size, max_blocks_per_seq, num_blocks, dtype, scale, out, cand[i], workspace,
+                         workspace_bytes, stream);
+    }
+    float ms = 0.f;
+    if (rc == PKV_OK && (cudaEventRecord(e1, st) != cudaSuccess || cudaEventSynchronize(e1) != cudaSuccess ||
+                         cudaEventElapsedTime(&ms, e0, e1) != cudaSuccess))
+      rc = PKV_ECUDA;
+    if (rc != PKV_OK) break;
+    ms /= reps;
+    if (times_ms && i < max_candidates) times_ms[i] = ms;
+    if (candidates && i < max_candidates) candidates[i] = cand[i];
+    if (best < 0 || ms < best_ms) {
+      best = cand[i];
+      best_ms = ms;
+    }
+  }
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  if (num_candidates) *num_candidates = nc;
+  if (rc != PKV_OK) return rc;
+  // leave `out` holding the result of the chosen partition size
+  rc = decode_impl(q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                   block_size, max_blocks_per_seq, num_blocks, dtype, scale, out, best, workspace, workspace_bytes,
+                   stream);
+  return rc != PKV_OK ? rc : best;
+}
+
+size_t paged_attn_decode_tune_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                             int block_size, int max_blocks_per_seq) {
+  // the smallest candidate partition needs the largest workspace
+  const long long max_ctx = (long long)max_blocks_per_seq * block_size;
+  if (max_ctx <= 0 || max_ctx > INT_MAX / 2) return (size_t)-1;
+  size_t most = paged_attn_decode_gqa_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                                     max_blocks_per_seq, 0);
+  if (most == (size_t)-1) return most;
+  for (int pt = 4096; pt >= 64; pt /= 2) {
+    if (pt % block_size || pt >= max_ctx) continue;
+    const size_t n = paged_attn_decode_gqa_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                                          max_blocks_per_seq, pt);
+    if (n == (size_t)-1) return n;
+    if (n > most) most = n;
+  }
+  return most;
+}
+
 int paged_attn_decode_gqa_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                            int block_size, int max_blocks_per_seq, int partition_tokens) {
   DecodePlan plan;

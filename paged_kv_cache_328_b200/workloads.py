@@ -420,7 +420,5 @@ def make(name, device="cpu", preappend=False, B=None):
 
 def last_block_waste(w):
     """Fraction of reserved slots left empty: only each sequence's last block is partial."""
-    ctx = w.context_lens.astype(np.int64)
-    blocks = -(-ctx // w.B)
-    reserved = int(blocks.sum()) * w.B
-    return 0.0 if reserved == 0 else 1.0 - int(ctx.sum()) / reserved
+    from .tuning import last_block_waste as waste
+    return waste(w.context_lens, w.B)
