@@ -125,7 +125,7 @@ int paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
 /*
  * Workspace bytes paged_attn_decode needs for these sizes and partition_tokens
  * (0 = the library's choice, resolved exactly as paged_attn_decode resolves it):
- * 16 + 4 * num_seqs * P rounded up to 16, plus 8 * S * H * P and
+ * 16 + 8 * num_seqs * P rounded up to 16, plus 8 * S * H * P and
  * 4 * S * H * P * head_dim (each rounded up to 16) when the call splits into
  * P > 1 partitions.
  * Returns (size_t)-1 for arguments paged_attn_decode would reject.  Pure host

@@ -3,11 +3,13 @@
 // Three kernels, launched back to back on one stream:
 //
 //  1. paged_decode_plan_kernel (one CTA): turns context_lens into a compact list
-//     of live (sequence, partition) work units, longest first when the list is
-//     short enough to sort in one CTA, and resets the unit counter.
+//     of live (sequence, partition) work units, each with its sequence's clamped
+//     context length, longest first when the list is short enough to sort in one
+//     CTA, and resets the unit counter.
 //  2. paged_decode_kernel (persistent, launched as a programmatic dependent of
-//     the plan so that its prologue overlaps it): every CTA takes units from the
-//     counter until none are left.  A unit is (sequence s, head h, partition p).
+//     the plan so that its prologue overlaps it): CTA b starts with unit b, then
+//     takes units from the counter until none are left.  A unit is (sequence s,
+//     head h, partition p).
 //     The CTA streams the unit's K and V rows through a ring of NS shared-memory
 //     stages:
 //       producer warp  follows the block table and issues one bulk (TMA-engine)
@@ -16,8 +18,9 @@
 //                      stage (unit, valid rows, first/last flags) and announces
 //                      the stage's bytes on its "full" mbarrier.  It reads the
 //                      table before waiting for a free stage and fetches the next
-//                      unit's list entry while streaming the current one, so the
-//                      ring does not drain between units.
+//                      unit's list entry (which carries the context length) while
+//                      streaming the current one, so the ring does not drain
+//                      between units.
 //       4 consumer warps   each 8-lane group takes one token at a time: a lane
 //                      owns D/8 dimensions, reads its 16-byte chunks of the K row
 //                      from shared memory, and the group reduces q.k with three
@@ -95,7 +98,7 @@ struct DecodeParams {
   float* out;         // [S][H][D]
   float* ws_acc;      // [S][H][max_parts][D]   (split only)
   float2* ws_ml;      // [S][H][max_parts]      (split only)
-  const uint32_t* units;  // (s << 16) | p for each live (sequence, partition)
+  const uint2* units;     // {(s << 16) | p, clamped context length} per live (sequence, partition)
   int* counters;          // [0] unit counter, [1] number of live (sequence, partition)
 };
 
@@ -122,6 +125,7 @@ constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 128;
 constexpr int kPlanBucketShift = 8;  // 256 tokens per bucket
 constexpr int kPlanSortMaxSeqs = 4096;  // sorted lists: num_seqs * partitions <= this
+static_assert(kPlanBuckets % 32 == 0, "the bucket scan gives every lane the same number of buckets");
 
 __device__ __forceinline__ int unit_bucket(int len) {
   return min(kPlanBuckets - 1, (len + (1 << kPlanBucketShift) - 1) >> kPlanBucketShift);
@@ -129,7 +133,7 @@ __device__ __forceinline__ int unit_bucket(int len) {
 
 __global__ void __launch_bounds__(kPlanThreads)
     paged_decode_plan_kernel(const int32_t* __restrict__ context_lens, int num_seqs, int max_ctx, int part_tokens,
-                             int sort, uint32_t* __restrict__ units, int* __restrict__ counters) {
+                             int sort, uint2* __restrict__ units, int* __restrict__ counters) {
   pdl_launch_dependents();
   __shared__ int scratch[kPlanBuckets];
   const int tid = threadIdx.x;
@@ -167,28 +171,46 @@ __global__ void __launch_bounds__(kPlanThreads)
         excl -= nfull;
         if (pass == 1) {
           const int at = scratch[key_full] + excl;
-          for (int j = 0; j < nfull; ++j) units[at + j] = ((uint32_t)s << 16) | (uint32_t)j;
+          for (int j = 0; j < nfull; ++j) units[at + j] = make_uint2(((uint32_t)s << 16) | (uint32_t)j, ctx);
         }
         __syncwarp();
         if (lane == 0 && tot > 0) scratch[key_full] += tot;
         __syncwarp();
         const int key = live ? unit_bucket(ctx - (n - 1) * part_tokens) : -1;
         const unsigned same = __match_any_sync(0xffffffffu, key);
-        if (live && pass == 1) units[scratch[key] + __popc(same & below)] = ((uint32_t)s << 16) | (uint32_t)(n - 1);
+        if (live && pass == 1)
+          units[scratch[key] + __popc(same & below)] = make_uint2(((uint32_t)s << 16) | (uint32_t)(n - 1), ctx);
         __syncwarp();
         if (live && (same & below) == 0) scratch[key] += __popc(same);
         __syncwarp();
       }
       if (pass == 0) {  // bucket start positions, longest bucket first
+        // lane l owns buckets 127-4l ... 124-4l; an exclusive scan over the lanes
+        // gives each bucket the count of all longer buckets
+        int c[kPlanBuckets / 32];
+        int mine = 0;
+#pragma unroll
+        for (int j = 0; j < kPlanBuckets / 32; ++j) {
+          c[j] = scratch[kPlanBuckets - 1 - (kPlanBuckets / 32) * lane - j];
+          mine += c[j];
+        }
+        int excl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, excl, o);
+          if (lane >= o) excl += v;
+        }
+        const int total = __shfl_sync(0xffffffffu, excl, 31);
+        excl -= mine;
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < kPlanBuckets / 32; ++j) {
+          scratch[kPlanBuckets - 1 - (kPlanBuckets / 32) * lane - j] = excl;
+          excl += c[j];
+        }
         if (lane == 0) {
-          int run = 0;
-          for (int k = kPlanBuckets - 1; k >= 0; --k) {
-            const int c = scratch[k];
-            scratch[k] = run;
-            run += c;
-          }
           counters[0] = 0;
-          counters[1] = run;
+          counters[1] = total;
         }
         __syncwarp();
       }
@@ -231,8 +253,9 @@ __global__ void __launch_bounds__(kPlanThreads)
   __syncthreads();
   int pos = scratch[warp] + incl - mine;
   for (int s = s0; s < s1; ++s) {
-    const int n = parts_of(clamp_ctx(context_lens[s], max_ctx), part_tokens);
-    for (int p = 0; p < n; ++p) units[pos++] = ((uint32_t)s << 16) | (uint32_t)p;
+    const int ctx = clamp_ctx(context_lens[s], max_ctx);
+    const int n = parts_of(ctx, part_tokens);
+    for (int p = 0; p < n; ++p) units[pos++] = make_uint2(((uint32_t)s << 16) | (uint32_t)p, ctx);
   }
 }
 
@@ -287,31 +310,34 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
     const int units_per_tile = TT / unit_rows;
     const long long total_units = (long long)prm.counters[1] * H;
 
-    auto describe = [&](int u, uint32_t sp) {
+    auto describe = [&](int u, uint2 e) {
       UnitDesc d{0, 0, 0, 0, 0, 1};
       if ((long long)u < total_units) {
-        d.s = (int)(sp >> 16);
-        d.p = (int)(sp & 0xffffu);
+        d.s = (int)(e.x >> 16);
+        d.p = (int)(e.x & 0xffffu);
         d.h = u - (u / H) * H;
-        const int ctx = clamp_ctx(prm.context_lens[d.s], max_ctx);
+        const int ctx = (int)e.y;  // clamped by the plan kernel
         d.t_begin = d.p * PT;
         d.t_end = min(ctx, d.t_begin + PT);
         d.n_parts = parts_of(ctx, PT);
       }
       return d;
     };
-
-    int u = 0;
-    if (lane == 0) u = atomicAdd(&prm.counters[0], 1);
-    u = __shfl_sync(0xffffffffu, u, 0);
-    UnitDesc cur = describe(u, (long long)u < total_units ? prm.units[u / H] : 0u);
+    // CTA b starts with unit b; later units come from the counter, offset by the grid
+    // size (lane 0 claims; the caller broadcasts the id when it needs it)
+    auto claim = [&]() { return lane == 0 ? (int)gridDim.x + atomicAdd(&prm.counters[0], 1) : 0; };
+    auto entry = [&](int u) {
+      return (long long)u < total_units ? __ldcg(prm.units + u / H) : make_uint2(0u, 0u);
+    };
+    int u = (int)blockIdx.x;
+    UnitDesc cur = describe(u, entry(u));
     int it = 0;  // stage iterations issued so far
     bool stop = false;
     while (!stop) {
       const bool done = (long long)u >= total_units;
+      const int u_next_lane0 = done ? 0 : claim();  // one unit ahead
       int u_next = 0;
-      if (!done && lane == 0) u_next = atomicAdd(&prm.counters[0], 1);
-      uint32_t sp_next = 0;
+      uint2 e_next = make_uint2(0u, 0u);
       const int n_tok = max(0, cur.t_end - cur.t_begin);
       const int n_tiles = done ? 1 : max(1, (n_tok + TT - 1) / TT);
       const int32_t* table = prm.block_tables + (size_t)cur.s * prm.max_blocks;
@@ -368,13 +394,13 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
                     Tr::kRowBytes, &full[stage], policy);
         }
         if (i == 0 && !done) {  // start fetching the next unit's list entry
-          u_next = __shfl_sync(0xffffffffu, u_next, 0);
-          if ((long long)u_next < total_units) sp_next = __ldcg(prm.units + u_next / H);
+          u_next = __shfl_sync(0xffffffffu, u_next_lane0, 0);
+          e_next = entry(u_next);
         }
       }
       if (done || stop) break;
       u = u_next;
-      cur = describe(u, sp_next);
+      cur = describe(u, e_next);
     }
     pdl_launch_dependents();  // this CTA takes no more units: the merge grid may be scheduled
     // Never leave with copies in flight into this CTA's shared memory.

@@ -11,7 +11,7 @@
 // Structure (persistent, one producer warp + 4 consumer warps, like the
 // multi-head kernel in decode.cuh):
 //  * unit = (sequence s, K/V head kvh, partition p); the plan kernel's list is
-//    reused, CTAs take units with an atomic counter.
+//    reused; CTA b starts with unit b, then takes units with an atomic counter.
 //  * producer: for every run of rows of one (block, K/V head) in the tile, two
 //    tensor-map TMA loads per 64 columns (K and V) into a 128-byte-swizzled
 //    stage; the G query rows are one bulk copy at a unit's first tile.
@@ -59,7 +59,7 @@ struct GqaParams {
   float* out;
   float* ws_acc;
   float2* ws_ml;
-  const uint32_t* units;
+  const uint2* units;  // {(s << 16) | p, clamped context length} per live (sequence, partition)
   int* counters;
 };
 
@@ -231,33 +231,36 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
     const uint32_t row_bytes = (uint32_t)(D * 2);
     const uint32_t run_bytes = (uint32_t)(unit_rows * 128);  // one 64-column box
 
-    auto describe = [&](int u, uint32_t sp) {
+    auto describe = [&](int u, uint2 e) {
       GqaUnit d{0, 0, 0, 0, 0, 0, 1, 0};
       if ((long long)u < total_units) {
-        d.s = (int)(sp >> 16);
-        d.p = (int)(sp & 0xffffu);
+        d.s = (int)(e.x >> 16);
+        d.p = (int)(e.x & 0xffffu);
         const int rem = u - (u / per_sp) * per_sp;
         d.kvh = rem / RT;
         d.rt = rem - d.kvh * RT;
-        d.ctx = clamp_ctx(prm.context_lens[d.s], max_ctx);
+        d.ctx = (int)e.y;  // clamped by the plan kernel
         d.t_begin = d.p * PT;
         d.t_end = min(d.ctx, d.t_begin + PT);
         d.n_parts = parts_of(d.ctx, PT);
       }
       return d;
     };
-
-    int u = 0;
-    if (lane == 0) u = atomicAdd(&prm.counters[0], 1);
-    u = __shfl_sync(0xffffffffu, u, 0);
-    GqaUnit cur = describe(u, (long long)u < total_units ? prm.units[u / per_sp] : 0u);
-    int it = 0;
+    // CTA b starts with unit b; later units come from the counter, offset by the grid
+    // size (lane 0 claims; the caller broadcasts the id when it needs it)
+    auto claim = [&]() { return lane == 0 ? (int)gridDim.x + atomicAdd(&prm.counters[0], 1) : 0; };
+    auto entry = [&](int u) {
+      return (long long)u < total_units ? __ldcg(prm.units + u / per_sp) : make_uint2(0u, 0u);
+    };
+    int u = (int)blockIdx.x;
+    GqaUnit cur = describe(u, entry(u));
+    int it = 0;  // stage iterations issued so far
     bool stop = false;
     while (!stop) {
       const bool done = (long long)u >= total_units;
+      const int u_next_lane0 = done ? 0 : claim();  // one unit ahead
       int u_next = 0;
-      if (!done && lane == 0) u_next = atomicAdd(&prm.counters[0], 1);
-      uint32_t sp_next = 0;
+      uint2 e_next = make_uint2(0u, 0u);
       const int n_tok = max(0, cur.t_end - cur.t_begin);
       const int n_tiles = done ? 1 : max(1, (n_tok + kGqaTile - 1) / kGqaTile);
       const int32_t* table = prm.block_tables + (size_t)cur.s * prm.max_blocks;
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
         const int tile_t0 = cur.t_begin + i * kGqaTile;
         const int u_t0 = tile_t0 + lane * unit_rows;
         const bool mine = !done && lane < units_per_tile && u_t0 < cur.t_end;
-        const int phys = mine ? __ldg(table + u_t0 / B) : -1;
+        const int phys = mine ? __ldg(table + u_t0 / B) : -1;  // u_t0 < ctx <= max_blocks * B
         if (it >= NS) {
           int ok = 1;
           if (lane == 0) ok = mbar_wait_bounded(&empty[stage], ((it / NS) - 1) & 1, abort_flag);
@@ -319,14 +322,14 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
           bulk_load(smem + Tr::kQOffset + stage * Tr::kQBytes + lane * row_bytes, qg + src, row_bytes, &full[stage],
                     policy);
         }
-        if (i == 0 && !done) {
-          u_next = __shfl_sync(0xffffffffu, u_next, 0);
-          if ((long long)u_next < total_units) sp_next = __ldcg(prm.units + u_next / per_sp);
+        if (i == 0 && !done) {  // start fetching the next unit's list entry
+          u_next = __shfl_sync(0xffffffffu, u_next_lane0, 0);
+          e_next = entry(u_next);
         }
       }
       if (done || stop) break;
       u = u_next;
-      cur = describe(u, sp_next);
+      cur = describe(u, e_next);
     }
     pdl_launch_dependents();
     if (lane == 0) {

@@ -90,7 +90,7 @@ int make_plan(int S, int H, int Hkv, int D, int B, int MB, int requested, Decode
   plan->sort = (long long)S * parts <= kSortedUnitsMax;
   size_t off = 16;  // counters[2] (+ padding)
   plan->off_units = off;
-  off += round16((size_t)S * parts * sizeof(uint32_t));
+  off += round16((size_t)S * parts * sizeof(uint2));
   if (plan->split) {
     plan->off_ml = off;
     off += round16((size_t)S * H * parts * sizeof(float2));
@@ -410,14 +410,14 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const i
   prm.out = out;
   prm.ws_acc = plan.split ? reinterpret_cast<float*>(ws + plan.off_acc) : nullptr;
   prm.ws_ml = plan.split ? reinterpret_cast<float2*>(ws + plan.off_ml) : nullptr;
-  prm.units = reinterpret_cast<const uint32_t*>(ws + plan.off_units);
+  prm.units = reinterpret_cast<const uint2*>(ws + plan.off_units);
   prm.counters = reinterpret_cast<int*>(ws);
 
   const int max_ctx = max_blocks_per_seq * block_size;
   int result = PKV_OK;
   pkv::paged_decode_plan_kernel<<<1, pkv::kPlanThreads, 0, st>>>(
       context_lens, num_seqs, max_ctx, plan.part_tokens, plan.sort ? 1 : 0,
-      reinterpret_cast<uint32_t*>(ws + plan.off_units), prm.counters);
+      reinterpret_cast<uint2*>(ws + plan.off_units), prm.counters);
   if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
   if (result == PKV_OK && use_gqa_kernel(num_heads, num_kv_heads, block_size, num_blocks, dtype)) {
     result = launch_tensor_core(q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1, num_heads,
@@ -480,13 +480,13 @@ int multi_query_impl(const void* q, const void* k_cache, const void* v_cache, co
   pkv::DecodeParams prm = {};
   prm.ws_acc = plan.split ? reinterpret_cast<float*>(ws + plan.off_acc) : nullptr;
   prm.ws_ml = plan.split ? reinterpret_cast<float2*>(ws + plan.off_ml) : nullptr;
-  prm.units = reinterpret_cast<const uint32_t*>(ws + plan.off_units);
+  prm.units = reinterpret_cast<const uint2*>(ws + plan.off_units);
   prm.counters = reinterpret_cast<int*>(ws);
   const int max_ctx = max_blocks_per_seq * block_size;
   int result = PKV_OK;
   pkv::paged_decode_plan_kernel<<<1, pkv::kPlanThreads, 0, st>>>(
       context_lens, num_seqs, max_ctx, plan.part_tokens, plan.sort ? 1 : 0,
-      reinterpret_cast<uint32_t*>(ws + plan.off_units), prm.counters);
+      reinterpret_cast<uint2*>(ws + plan.off_units), prm.counters);
   if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
   if (result == PKV_OK)
     result = launch_tensor_core(q, k_cache, v_cache, block_tables, context_lens, num_seqs, q_len, num_heads,

@@ -58,11 +58,11 @@ def test_strerror_and_version(lib):
 
 
 def test_workspace_size_layout(lib):
-    # no split: counters (16) + 4 bytes per sequence rounded to 16
-    assert _lib.workspace_size(256, 40, 128, 16, 128, 2048) == 16 + 1024
+    # no split: counters (16) + an 8-byte unit entry per sequence, rounded to 16
+    assert _lib.workspace_size(256, 40, 128, 16, 128, 2048) == 16 + 2048
     # split into 64 partitions of 512 tokens: + m/l and acc per partition
     n = _lib.workspace_size(8, 40, 128, 16, 2048, 512)
-    assert n == 16 + 8 * 64 * 4 + 8 * 40 * 64 * 8 + 8 * 40 * 64 * 128 * 4
+    assert n == 16 + 8 * 64 * 8 + 8 * 40 * 64 * 8 + 8 * 40 * 64 * 128 * 4
     assert _lib.partition_tokens(8, 40, 128, 16, 2048, 512) == 512
     # the library's own choice splits long contexts into 512-token partitions
     assert _lib.partition_tokens(8, 40, 128, 16, 2048, 0) == 512
