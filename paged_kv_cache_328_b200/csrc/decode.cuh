@@ -281,7 +281,6 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int H = prm.num_heads;
-  const int max_ctx = prm.max_blocks * prm.block_size;
   const int PT = prm.part_tokens;
 
   if (threadIdx.x == 0) {

@@ -199,7 +199,6 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_gqa_kernel(const 
   const int G = prm.group;
   const int Lq = prm.q_len;
   const int RT = prm.row_tiles;
-  const int max_ctx = prm.max_blocks * prm.block_size;
   const int PT = prm.part_tokens;
 
   if (threadIdx.x == 0) {

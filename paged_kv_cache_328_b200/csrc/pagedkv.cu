@@ -170,14 +170,31 @@ int launch_decode(const pkv::DecodeParams& prm, long long max_units, cudaStream_
 }
 
 // Tile sizes: every stage holds 32 KB of K+V (64 rows of 256 bytes for 16-bit
-// D=128); three stages per CTA, two CTAs per SM.
+// D=128).  16-bit K/V with at least kShallowRingUnits (sequence, head,
+// partition) units runs two stages per CTA and three CTAs per SM; fewer units
+// run three stages and two CTAs per SM.  The shallow ring keeps the same bytes in
+// flight per SM but gives it three independent unit streams, so the SM crosses
+// unit boundaries (a block-table and list-entry round trip each) more often in
+// parallel, and more sequences that share prefix blocks run at the same time and
+// meet in L2.  With few units the longest one becomes the critical path, and a
+// CTA's share of HBM bandwidth shrinks with every extra CTA.  Measured on B200
+// (bf16/fp16, D=128, B=16): three CTAs per SM are 1-4% faster for batch 64-256
+// OPT-13B layers, 17% at B=8, 22% for the shared-prefix sampling batch and 6%
+// for a batch-128 LLaMA-7B layer; 8-10% slower at 1280 and 2048 units.
+constexpr long long kShallowRingUnits = 8 * kRefCtas;
+
 template <int D>
 int dispatch_decode(pkv_dtype dt, const pkv::DecodeParams& prm, long long max_units, cudaStream_t st) {
   constexpr int kTT16 = 16384 / (D * 2);
   constexpr int kTT32 = 16384 / (D * 4);
+  const bool shallow = max_units >= kShallowRingUnits;
   switch (dt) {
-    case PKV_F16: return launch_decode<__half, D, kTT16, 3>(prm, max_units, st);
-    case PKV_BF16: return launch_decode<__nv_bfloat16, D, kTT16, 3>(prm, max_units, st);
+    case PKV_F16:
+      return shallow ? launch_decode<__half, D, kTT16, 2>(prm, max_units, st)
+                     : launch_decode<__half, D, kTT16, 3>(prm, max_units, st);
+    case PKV_BF16:
+      return shallow ? launch_decode<__nv_bfloat16, D, kTT16, 2>(prm, max_units, st)
+                     : launch_decode<__nv_bfloat16, D, kTT16, 3>(prm, max_units, st);
     case PKV_F32: return launch_decode<float, D, kTT32, 3>(prm, max_units, st);
   }
   return PKV_EDTYPE;

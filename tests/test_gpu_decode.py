@@ -97,6 +97,27 @@ def test_small_ragged(dev, dtype, D, B):
     no_device_error(dev)
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("B", [8, 16, 128])
+@pytest.mark.parametrize("H", [36, 37])
+def test_ring_depth_boundary_ragged(dev, dtype, D, B, H):
+    # 16-bit decode runs a two-stage ring (three CTAs per SM) from 8 x 296 = 2368
+    # (sequence, head, partition) units up, a three-stage ring below: 64 x 36 units
+    # unsplit run the deep ring, 64 x 37 and every split run the shallow one
+    ctx = np.array([RAGGED[i % len(RAGGED)] for i in range(64)])
+    mb = -(-max(RAGGED) // B) + 1
+    w = wl.build_paged(ctx, H=H, D=D, B=B, dtype=dtype, seed=300 + H + D + B, device=dev, max_blocks=mb)
+    ix = dev_indices(w, dev)
+    want = full_oracle(w)
+    for pt in sorted({0, max(B, 64), 256, mb * B}):
+        got = decode(w, ix, pt=pt).cpu().numpy()
+        assert np.all(np.isfinite(got)), pt
+        assert max_err(got, want) <= TOL[dtype], (pt, max_err(got, want))
+        assert np.all(got[ctx == 0] == 0.0)
+    no_device_error(dev)
+
+
 def test_one_token_contexts_return_v_exactly(dev):
     for dtype in ("f32", "f16", "bf16"):
         w = wl.build_paged([1] * 7, H=4, D=128, B=16, dtype=dtype, seed=7, device=dev)
