@@ -467,7 +467,8 @@ def run_gpu(a, rank, world, local_rank):
     value, _ = job_throughput(kv_bytes, [ms_step] * world)
     peak, peak_src = measured_peaks()
     achieved = kv_bytes / (dec_ms * 1e-3) / 1e9
-    wkey = f"{w.name}" + (f"_pt{pt}" if pt else "")
+    # the traffic record belongs to one kernel: multi-token queries run another one
+    wkey = f"{w.name}" + (f"_pt{pt}" if pt else "") + (f"_L{Lq}" if Lq > 1 else "")
     result = {
         "metric": METRIC,
         "value": round(value, 1),

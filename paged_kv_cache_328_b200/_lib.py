@@ -116,7 +116,7 @@ def _check(rc, where):
 def _cuda(t, name, dtypes=None):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != "cuda":
+    if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (got {t.device}); there is no CPU path")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
@@ -129,6 +129,15 @@ def _stream(device, stream):
     if stream is None:
         stream = torch.cuda.current_stream(device)
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _call(fn, args, device, stream):
+    """fn(*args, stream) with `device` current; the device is switched only when it is not
+    already the current one (entering a device context costs more than the launch)."""
+    if device.index is None or device.index == torch.cuda.current_device():
+        return fn(*args, _stream(device, stream))
+    with torch.cuda.device(device):
+        return fn(*args, _stream(device, stream))
 
 
 def workspace_size(num_seqs, num_heads, head_dim, block_size, max_blocks, partition_tokens=0):
@@ -201,11 +210,10 @@ def paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale, ou
             S, H, Hkv, D, B, block_tables.shape[1], NB, dt, float(scale),
             _cuda(out, "out", (torch.float32,)), int(partition_tokens),
             _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size())
-    with torch.cuda.device(q.device):
-        if Hkv == H:
-            rc = lib.paged_attn_decode(*args[:6], *args[7:], _stream(q.device, stream))
-        else:
-            rc = lib.paged_attn_decode_gqa(*args, _stream(q.device, stream))
+    if Hkv == H:
+        rc = _call(lib.paged_attn_decode, args[:6] + args[7:], q.device, stream)
+    else:
+        rc = _call(lib.paged_attn_decode_gqa, args, q.device, stream)
     _check(rc, "paged_attn_decode" if Hkv == H else "paged_attn_decode_gqa")
     return out
 
@@ -224,8 +232,7 @@ def kv_cache_append(k, v, k_cache, v_cache, slot_mapping, stream=None):
     args = (_cuda(k, "k", DTYPE_CODE), _cuda(v, "v", DTYPE_CODE), _cuda(k_cache, "k_cache"),
             _cuda(v_cache, "v_cache"), _cuda(slot_mapping, "slot_mapping", (torch.int64,)),
             T, H, D, B, NB, DTYPE_CODE[k_cache.dtype])
-    with torch.cuda.device(k_cache.device):
-        rc = lib.kv_cache_append(*args, _stream(k_cache.device, stream))
+    rc = _call(lib.kv_cache_append, args, k_cache.device, stream)
     _check(rc, "kv_cache_append")
 
 
@@ -240,8 +247,7 @@ def kv_block_copy(k_cache, v_cache, src_dst_pairs, stream=None):
     args = (_cuda(k_cache, "k_cache", DTYPE_CODE), _cuda(v_cache, "v_cache", DTYPE_CODE),
             _cuda(src_dst_pairs, "src_dst_pairs", (torch.int64,)), src_dst_pairs.shape[0],
             H, D, B, NB, DTYPE_CODE[k_cache.dtype])
-    with torch.cuda.device(k_cache.device):
-        rc = lib.kv_block_copy(*args, _stream(k_cache.device, stream))
+    rc = _call(lib.kv_block_copy, args, k_cache.device, stream)
     _check(rc, "kv_block_copy")
 
 
@@ -256,8 +262,7 @@ def paged_kv_gather(cache, block_table_row, context_len, out=None, stream=None):
         raise ValueError("out must be [H, context_len, D] in the cache dtype")
     args = (_cuda(cache, "cache", DTYPE_CODE), _cuda(block_table_row, "block_table_row", (torch.int32,)),
             int(context_len), H, D, B, NB, DTYPE_CODE[cache.dtype], _cuda(out, "out"))
-    with torch.cuda.device(cache.device):
-        rc = lib.paged_kv_gather(*args, _stream(cache.device, stream))
+    rc = _call(lib.paged_kv_gather, args, cache.device, stream)
     _check(rc, "paged_kv_gather")
     return out
 
@@ -267,8 +272,7 @@ def get_device_error(device=None, stream=None):
     lib = load()
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     reason = ctypes.c_int(0)
-    with torch.cuda.device(dev):
-        rc = lib.pkv_get_device_error(_stream(dev, stream), ctypes.byref(reason))
+    rc = _call(lambda st: lib.pkv_get_device_error(st, ctypes.byref(reason)), (), dev, stream)
     return rc, reason.value
 
 
@@ -301,8 +305,7 @@ def paged_attn_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, s
             _cuda(context_lens, "context_lens", (torch.int32,)),
             S, H, D, B, block_tables.shape[1], NB, DTYPE_CODE[k_cache.dtype], float(scale),
             _cuda(out, "out", (torch.float32,)), int(partition_tokens))
-    with torch.cuda.device(q.device):
-        rc = lib.paged_attn_decode_noalloc(*args, _stream(q.device, stream))
+    rc = _call(lib.paged_attn_decode_noalloc, args, q.device, stream)
     _check(rc, "paged_attn_decode_noalloc")
     return out
 
@@ -335,8 +338,7 @@ def paged_attn_multi_query(q, k_cache, v_cache, block_tables, context_lens, scal
             S, Lq, H, Hkv, D, B, block_tables.shape[1], NB, DTYPE_CODE[k_cache.dtype], float(scale),
             _cuda(out, "out", (torch.float32,)), int(partition_tokens),
             _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size())
-    with torch.cuda.device(q.device):
-        rc = lib.paged_attn_multi_query(*args, _stream(q.device, stream))
+    rc = _call(lib.paged_attn_multi_query, args, q.device, stream)
     _check(rc, "paged_attn_multi_query")
     return out
 
@@ -357,8 +359,7 @@ def kv_blocks_to_host(k_cache, v_cache, block_ids, host_k, host_v, stream=None):
     args = (_cuda(k_cache, "k_cache", DTYPE_CODE), _cuda(v_cache, "v_cache", DTYPE_CODE),
             _cuda(block_ids, "block_ids", (torch.int64,)), n, _host_pinned(host_k, "host_k"),
             _host_pinned(host_v, "host_v"), H, D, B, NB, DTYPE_CODE[k_cache.dtype])
-    with torch.cuda.device(k_cache.device):
-        rc = lib.kv_blocks_to_host(*args, _stream(k_cache.device, stream))
+    rc = _call(lib.kv_blocks_to_host, args, k_cache.device, stream)
     _check(rc, "kv_blocks_to_host")
 
 
@@ -372,8 +373,7 @@ def kv_blocks_from_host(host_k, host_v, k_cache, v_cache, block_ids, stream=None
     args = (_host_pinned(host_k, "host_k"), _host_pinned(host_v, "host_v"),
             _cuda(k_cache, "k_cache", DTYPE_CODE), _cuda(v_cache, "v_cache", DTYPE_CODE),
             _cuda(block_ids, "block_ids", (torch.int64,)), n, H, D, B, NB, DTYPE_CODE[k_cache.dtype])
-    with torch.cuda.device(k_cache.device):
-        rc = lib.kv_blocks_from_host(*args, _stream(k_cache.device, stream))
+    rc = _call(lib.kv_blocks_from_host, args, k_cache.device, stream)
     _check(rc, "kv_blocks_from_host")
 
 
@@ -488,8 +488,7 @@ def tune_partition_tokens(q, k_cache, v_cache, block_tables, context_lens, scale
             _cuda(block_tables, "block_tables", (torch.int32,)), _cuda(context_lens, "context_lens", (torch.int32,)),
             S, H, Hkv, D, B, MB, NB, DTYPE_CODE[k_cache.dtype], float(scale), _cuda(out, "out", (torch.float32,)),
             ws.data_ptr(), n, int(reps), times, cands, 8, ctypes.byref(nc))
-    with torch.cuda.device(q.device):
-        rc = lib.paged_attn_decode_tune(*args, _stream(q.device, stream))
+    rc = _call(lib.paged_attn_decode_tune, args, q.device, stream)
     if rc < 0:
         raise PagedKVError(rc, "paged_attn_decode_tune")
     return rc, {cands[i]: times[i] for i in range(nc.value)}
