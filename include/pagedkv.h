@@ -360,6 +360,20 @@ int pkv_bm_swap_out(pkv_block_manager* bm, int64_t seq, int64_t* blocks, int max
 int pkv_bm_swap_in(pkv_block_manager* bm, int64_t seq, int64_t* blocks, int max_blocks, int* n_blocks);
 
 /*
+ * pkv_selftest_wait_timeout - exercise the bounded-wait path that every pipeline
+ * wait in the attention kernels uses (no counterpart on the pages: failure
+ * detection for the library itself).  Launches one CTA on `stream` whose thread 0
+ * waits on a fresh shared-memory mbarrier that nothing arrives on, bounded by
+ * `limit_cycles` SM clock cycles (1 ... 2e9, the kernels' own bound); the wait runs
+ * out, the kernel records PKV_DEV_WAIT_TIMEOUT in the device error word and returns
+ * normally, so the context stays usable.  Synchronises the stream.  Returns 1 when
+ * the wait ran out, 0 if it completed (it cannot), PKV_EINVAL for a limit out of
+ * range (checked on the host, nothing launched) or PKV_ECUDA.  Read and clear the
+ * recorded reason with pkv_get_device_error.
+ */
+int pkv_selftest_wait_timeout(long long limit_cycles, void* stream);
+
+/*
  * pkv_get_device_error - synchronise `stream`, read and clear the device error
  * word of the current device.  Returns PKV_OK when it was clear, PKV_ETIMEOUT when
  * it records PKV_DEV_WAIT_TIMEOUT, PKV_EDEVICE for any other reason, PKV_ECUDA if

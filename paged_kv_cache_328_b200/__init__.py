@@ -34,6 +34,7 @@ from ._lib import (  # noqa: F401
     paged_attn_multi_query,
     paged_kv_gather,
     partition_tokens,
+    selftest_wait_timeout,
     strerror,
     tune_partition_tokens,
     workspace_size,

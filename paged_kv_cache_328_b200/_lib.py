@@ -50,6 +50,7 @@ SIGNATURES = {
                                                                      _c_size_t, _c_int, _c_void_p, _c_void_p,
                                                                      _c_int, ctypes.POINTER(_c_int), _c_void_p]),
     "paged_attn_decode_tune_workspace_size": (_c_size_t, [_c_int] * 6),
+    "pkv_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _c_void_p]),
     "kv_blocks_to_host": (_c_int, [_c_void_p] * 3 + [_c_int] + [_c_void_p] * 2 + [_c_int] * 5 + [_c_void_p]),
     "kv_blocks_from_host": (_c_int, [_c_void_p] * 5 + [_c_int] * 6 + [_c_void_p]),
     "pkv_bm_create": (_c_void_p, [_c_int, _c_int, _c_void_p]),
@@ -265,6 +266,17 @@ def paged_kv_gather(cache, block_table_row, context_len, out=None, stream=None):
     rc = _call(lib.paged_kv_gather, args, cache.device, stream)
     _check(rc, "paged_kv_gather")
     return out
+
+
+def selftest_wait_timeout(limit_cycles=20_000_000, device=None, stream=None):
+    """Run the bounded-wait self-test kernel: True when its deliberately stalled wait ran out
+    (the device error word then holds PKV_DEV_WAIT_TIMEOUT; read it with get_device_error)."""
+    lib = load()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    rc = _call(lambda st: lib.pkv_selftest_wait_timeout(int(limit_cycles), st), (), dev, stream)
+    if rc < 0:
+        raise PagedKVError(rc, "pkv_selftest_wait_timeout")
+    return rc == 1
 
 
 def get_device_error(device=None, stream=None):

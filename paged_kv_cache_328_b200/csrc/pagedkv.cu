@@ -807,6 +807,23 @@ int pkv_get_device_error(void* stream, int* reason) {
   return word == PKV_DEV_WAIT_TIMEOUT ? PKV_ETIMEOUT : PKV_EDEVICE;
 }
 
+int pkv_selftest_wait_timeout(long long limit_cycles, void* stream) {
+  if (limit_cycles <= 0 || limit_cycles > pkv::kWaitLimitCycles) return PKV_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int minus_one = -1;
+  if (cudaMemcpyToSymbolAsync(pkv::g_selftest_waited_out, &minus_one, sizeof(int), 0, cudaMemcpyHostToDevice, st) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  pkv::wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(limit_cycles);
+  if (cudaGetLastError() != cudaSuccess) return PKV_ECUDA;
+  int waited_out = -1;
+  if (cudaMemcpyFromSymbolAsync(&waited_out, pkv::g_selftest_waited_out, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return PKV_ECUDA;
+  return waited_out == 1 ? 1 : (waited_out == 0 ? 0 : PKV_ECUDA);
+}
+
 const char* pkv_strerror(int code) {
   switch (code) {
     case PKV_OK: return "success";

@@ -65,13 +65,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Waits for the phase with the given parity to complete.  Returns false if the
 // CTA-wide abort flag is raised or the wait exceeds kWaitLimitCycles.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  long long limit_cycles = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) return false;
+    if (clock64() - t0 > limit_cycles) return false;
+  }
+}
+
+// Self-test of the bounded wait: one thread waits on a barrier that nothing
+// arrives on; the wait must give up after `limit_cycles` and record
+// PKV_DEV_WAIT_TIMEOUT, after which the kernel returns normally.
+__device__ int g_selftest_waited_out = 0;
+
+__global__ void wait_timeout_selftest_kernel(long long limit_cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait_bounded(&bar, 0, &abort_flag, limit_cycles);
+    if (!ok) flag_error(PKV_DEV_WAIT_TIMEOUT);
+    g_selftest_waited_out = ok ? 0 : 1;
   }
 }
 

@@ -152,3 +152,9 @@ def test_binding_refuses_cpu_tensors(lib):
         _lib.paged_attn_decode(q, kc, kc, torch.zeros(1, 1, dtype=torch.int32),
                                torch.zeros(1, dtype=torch.int32), 1.0,
                                workspace=torch.zeros(64, dtype=torch.uint8))
+
+
+def test_wait_selftest_rejects_limits_on_host(lib):
+    assert lib.pkv_selftest_wait_timeout(0, None) == PKV_EINVAL
+    assert lib.pkv_selftest_wait_timeout(-5, None) == PKV_EINVAL
+    assert lib.pkv_selftest_wait_timeout(2_000_000_001, None) == PKV_EINVAL

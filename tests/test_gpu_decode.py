@@ -118,6 +118,22 @@ def test_ring_depth_boundary_ragged(dev, dtype, D, B, H):
     no_device_error(dev)
 
 
+def test_plan_sort_many_sequences(dev):
+    # 1500 sequences: the plan's sorted path with several runs of 32 sequences per warp,
+    # unsplit (1500 entries) and with full + last 512-token partitions (3000 entries);
+    # 256-token partitions (4500 entries) take the unsorted path
+    rng = np.random.default_rng(77)
+    ctx = rng.integers(0, 601, 1500)
+    w = wl.build_paged(ctx, H=2, D=64, B=16, dtype="f16", seed=77, device=dev, max_blocks=38)
+    ix = dev_indices(w, dev)
+    want = full_oracle(w)
+    for pt in (0, 512, 256):
+        got = decode(w, ix, pt=pt).cpu().numpy()
+        assert max_err(got, want) <= TOL["f16"], pt
+        assert np.all(got[ctx == 0] == 0.0)
+    no_device_error(dev)
+
+
 def test_one_token_contexts_return_v_exactly(dev):
     for dtype in ("f32", "f16", "bf16"):
         w = wl.build_paged([1] * 7, H=4, D=128, B=16, dtype=dtype, seed=7, device=dev)
