@@ -1,0 +1,648 @@
+// Paged attention for many query rows per K/V head on the 5th-generation tensor
+// cores (tcgen05, sm_100a): the verify pass of speculative decoding and chunked
+// prefill, where Lq new tokens of a sequence (times G query heads per K/V head)
+// attend its paged context ("vLLM PagedAttention and continuous batching",
+// section 5 on chunked prefill; the multi-token generalisation of the decode in
+// "PagedAttention - Efficient Memory Management for LLM Serving with vLLM",
+// section "Method (PagedAttention + vLLM)").
+//
+// A unit is (sequence s, K/V head kvh, row tile rt, partition p) from the plan
+// kernel's list.  Its R <= 128 query rows (row r = query token rt*Tq + r/G, query
+// head kvh*G + r%G) form the M = 128 operand of every MMA; the K/V context streams
+// through 64-token tiles:
+//
+//   S = Q K^T           tcgen05.mma  M=128 N=64  K=D   (Q and the K tile from shared memory)
+//   P = 2^(S*scale - m) four softmax warps, one row per thread, S read from tensor memory
+//   O += P V            tcgen05.mma  M=128 N=D   K=64  (P from shared memory, V as an MN-major operand)
+//
+// S (double-buffered, 2 x 64 columns) and O (D columns) live in tensor memory.
+// P is split into a 16-bit high part and the 16-bit rounding of the rest, and both
+// are multiplied (with P rounded to 16 bits alone the error exceeds 2e-3).  O is
+// rescaled only when a row's running maximum grows by more than 2^8 (the partial
+// sums stay exact in fp32; the final division uses the same reference maximum).
+//
+// Warp roles (one CTA per SM, persistent over the unit list):
+//   warp 0     producer: the unit's query tile (one 4-D TMA box per 64 columns) and
+//              the K/V tiles (2-D TMA boxes per (block, K/V head) run, 128-byte swizzle);
+//   warp 1     allocates / frees the tensor memory; its lane 0 issues every MMA and
+//              commits completion to mbarriers;
+//   warps 2-5  softmax and epilogue; warp w reads tensor-memory lanes 32*(w%4) ...
+//
+// Every mbarrier wait is bounded (kWaitLimitCycles) and checks the CTA abort flag;
+// before the tensor memory is freed the MMA thread waits for all its MMAs.
+#pragma once
+
+#include "decode_gqa.cuh"
+
+namespace pkv {
+
+constexpr int kTcRows = 128;          // M: query rows per tile = tensor-memory lanes
+constexpr int kTcTile = 64;           // tokens per K/V tile
+constexpr int kTcStages = 3;
+constexpr int kTcThreads = 6 * 32;    // producer, MMA, four softmax warps
+constexpr int kTcTmemCols = 256;      // S[2] at columns 0 and 64, O at column 128
+constexpr float kTcRescaleLog2 = 8.0f;
+
+struct TcParams {
+  CUtensorMap tmap_k;  // 2-D view [NB*Hkv*B rows][D] of the K pool, box {64, unit_rows}, 128B swizzle
+  CUtensorMap tmap_v;
+  CUtensorMap tmap_q;  // 4-D view [S][Lq][Hq][D] of q, box {64, G, Tq, 1}, 128B swizzle
+  const int32_t* block_tables;
+  int num_heads;       // Hq
+  int num_kv_heads;    // Hkv
+  int group;           // G
+  int q_len;           // Lq
+  int tq_per_tile;     // Tq = floor(128 / G) query tokens per row tile
+  int row_tiles;       // ceil(Lq / Tq)
+  int block_size;
+  int max_blocks;
+  int num_blocks;
+  float scale_log2;
+  int part_tokens;
+  int max_parts;
+  float* out;          // [S][Lq][Hq][D]
+  float* ws_acc;
+  float2* ws_ml;
+  const uint2* units;
+  int* counters;
+};
+
+template <int D>
+struct TcTraits {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kSlabBytes = kTcTile * 128;          // 64 tokens x 64 columns
+  static constexpr int kTileBytes = kHalves * kSlabBytes;   // K (or V) part of a stage
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kQSlabBytes = kTcRows * 128;         // 128 rows x 64 columns
+  static constexpr int kQOffset = kTcStages * kStageBytes;
+  static constexpr int kPBytes = kTcRows * kTcTile * 2;     // 128 rows x 64 tokens, one slab
+  static constexpr int kPOffset = kQOffset + kHalves * kQSlabBytes;  // P high, then P low
+  static constexpr int kHdrOffset = kPOffset + 2 * kPBytes;          // two int4 per stage
+  static constexpr int kBarOffset = kHdrOffset + kTcStages * 32;
+  // full[NS], empty[NS], q_full, q_empty, s_full[2], s_free[2], p_full, o_done, drain
+  static constexpr int kNumBars = 2 * kTcStages + 9;
+  static constexpr int kTmemSlotOffset = kBarOffset + kNumBars * 8;
+  static constexpr int kAbortOffset = kTmemSlotOffset + 8;
+  static constexpr int kSmemBytes = kAbortOffset + 8;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;      // the base is rounded up to 1024 bytes
+  static constexpr uint32_t kOCol = 128;
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static_assert(kQOffset % 1024 == 0 && kPOffset % 1024 == 0, "swizzle atoms are 1024-byte aligned");
+  static_assert(kSmemAlloc <= 227 * 1024, "shared memory per CTA");
+};
+
+// ---- tcgen05 helpers ---------------------------------------------------------
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: start, leading
+// and stride byte offsets in 16-byte units, version 1, layout type 2).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Operand format code of kind::f16 (fp16 = 0, bf16 = 1).
+template <typename T>
+struct TcFormat;
+template <>
+struct TcFormat<__half> {
+  static constexpr uint32_t kCode = 0;
+};
+template <>
+struct TcFormat<__nv_bfloat16> {
+  static constexpr uint32_t kCode = 1;
+};
+
+// Instruction descriptor for kind::f16 with fp32 accumulation: A and B of one type
+// (both fp16 or both bf16), A K-major, B K-major or MN-major, M x N.
+template <typename T>
+__host__ __device__ constexpr uint32_t umma_idesc(int M, int N, bool b_mn_major) {
+  return (1u << 4) | (TcFormat<T>::kCode << 7) | (TcFormat<T>::kCode << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 16 consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Wait for this thread's tensor-memory loads, then pin the loaded registers after
+// the wait (the empty asm redefines them, so no use is scheduled above it).
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]));
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                            uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_addr(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+template <typename T>
+__device__ __forceinline__ float round16(float a);
+template <>
+__device__ __forceinline__ float round16<__half>(float a) {
+  return __half2float(__float2half_rn(a));
+}
+template <>
+__device__ __forceinline__ float round16<__nv_bfloat16>(float a) {
+  return __bfloat162float(__float2bfloat16_rn(a));
+}
+
+struct TcUnit {
+  int s, kvh, rt, p, t_begin, t_end, n_parts, ctx;
+};
+
+// grid = min(#SMs, units); block = kTcThreads; one CTA per SM (shared memory).
+template <typename T, int D>
+__global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(const __grid_constant__ TcParams prm) {
+  using Tr = TcTraits<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::kBarOffset);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kTcStages;
+  uint64_t* q_full = bars + 2 * kTcStages;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* s_full = q_full + 2;  // [2]
+  uint64_t* s_free = q_full + 4;  // [2]
+  uint64_t* p_full = q_full + 6;
+  uint64_t* o_done = q_full + 7;
+  uint64_t* drain = q_full + 8;
+  int4* hdr = reinterpret_cast<int4*>(smem + Tr::kHdrOffset);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::kTmemSlotOffset);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Tr::kAbortOffset);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int Hkv = prm.num_kv_heads;
+  const int G = prm.group;
+  const int Tq = prm.tq_per_tile;
+  const int RT = prm.row_tiles;
+  const int PT = prm.part_tokens;
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(&s_free[0], 4);
+    mbar_init(&s_free[1], 4);
+    mbar_init(p_full, 4);
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // query rows that no TMA box covers (rows >= G * Tq) must read as zero
+  for (int i = threadIdx.x; i < Tr::kHalves * Tr::kQSlabBytes / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem + Tr::kQOffset)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                 "r"(kTcTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait_primary();
+
+  const int per_sp = Hkv * RT;  // units per (sequence, partition)
+  const long long total_units = (long long)prm.counters[1] * per_sp;
+
+  if (warp == 0) {
+    // ------------------------------- producer -------------------------------
+    const uint64_t policy = l2_evict_first();
+    const int B = prm.block_size;
+    const int unit_rows = min(B, kTcTile);
+    const int units_per_tile = kTcTile / unit_rows;
+    const uint32_t run_bytes = (uint32_t)(unit_rows * 128);
+    const uint32_t q_bytes = (uint32_t)(Tr::kHalves * 128 * G * Tq);
+
+    auto describe = [&](int u, uint2 e) {
+      TcUnit d{0, 0, 0, 0, 0, 0, 1, 0};
+      if ((long long)u < total_units) {
+        d.s = (int)(e.x >> 16);
+        d.p = (int)(e.x & 0xffffu);
+        const int rem = u - (u / per_sp) * per_sp;
+        d.kvh = rem / RT;
+        d.rt = rem - d.kvh * RT;
+        d.ctx = (int)e.y;
+        d.t_begin = d.p * PT;
+        d.t_end = min(d.ctx, d.t_begin + PT);
+        d.n_parts = parts_of(d.ctx, PT);
+      }
+      return d;
+    };
+    auto claim = [&]() { return lane == 0 ? (int)gridDim.x + atomicAdd(&prm.counters[0], 1) : 0; };
+    auto entry = [&](int u) {
+      return (long long)u < total_units ? __ldcg(prm.units + u / per_sp) : make_uint2(0u, 0u);
+    };
+
+    int u = (int)blockIdx.x;
+    TcUnit cur = describe(u, entry(u));
+    int it = 0;  // tiles issued
+    int nu = 0;  // query tiles issued
+    bool stop = false;
+    while (!stop) {
+      const bool done = (long long)u >= total_units;
+      const int u_next_lane0 = done ? 0 : claim();
+      int u_next = 0;
+      uint2 e_next = make_uint2(0u, 0u);
+      if (!done) {
+        // the previous unit's S products must be done reading the query tile
+        int ok = 1;
+        if (nu > 0 && lane == 0) ok = mbar_wait_bounded(q_empty, (nu - 1) & 1, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) {
+            flag_error(PKV_DEV_WAIT_TIMEOUT);
+            *abort_flag = 1;
+          }
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full, q_bytes);
+#pragma unroll
+          for (int hf = 0; hf < Tr::kHalves; ++hf)
+            tma_load_4d(smem + Tr::kQOffset + hf * Tr::kQSlabBytes, &prm.tmap_q, hf * 64, cur.kvh * G,
+                        cur.rt * Tq, cur.s, q_full, policy);
+        }
+        ++nu;
+      }
+      const int n_tok = max(0, cur.t_end - cur.t_begin);
+      const int n_tiles = done ? 1 : max(1, (n_tok + kTcTile - 1) / kTcTile);
+      const int32_t* table = prm.block_tables + (size_t)cur.s * prm.max_blocks;
+
+      for (int i = 0; i < n_tiles; ++i, ++it) {
+        const int stage = it % kTcStages;
+        const int tile_t0 = cur.t_begin + i * kTcTile;
+        const int u_t0 = tile_t0 + lane * unit_rows;
+        const bool mine = !done && lane < units_per_tile && u_t0 < cur.t_end;
+        const int phys = mine ? __ldg(table + u_t0 / B) : -1;  // u_t0 < ctx <= max_blocks * B
+        if (it >= kTcStages) {
+          int ok = 1;
+          if (lane == 0) ok = mbar_wait_bounded(&empty[stage], ((it / kTcStages) - 1) & 1, abort_flag);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) {
+            if (lane == 0) {
+              flag_error(PKV_DEV_WAIT_TIMEOUT);
+              *abort_flag = 1;
+            }
+            stop = true;
+            break;
+          }
+        }
+        const int n_valid = done ? 0 : max(0, min(kTcTile, cur.t_end - tile_t0));
+        bool load = false;
+        if (mine) {
+          if (phys >= 0 && phys < prm.num_blocks)
+            load = true;
+          else
+            flag_error(PKV_DEV_BLOCK_ID);
+        }
+        const unsigned loads = __ballot_sync(0xffffffffu, load);
+        if (lane == 0) {
+          const int flags = done ? kTileEnd : ((i == 0 ? kTileFirst : 0) | (i == n_tiles - 1 ? kTileLast : 0));
+          hdr[2 * stage] = make_int4(cur.s, cur.kvh | (cur.rt << 16), cur.p | (cur.n_parts << 16),
+                                     n_valid | (flags << 16));
+          hdr[2 * stage + 1] = make_int4(tile_t0, cur.ctx, 0, 0);
+          mbar_arrive_expect_tx(&full[stage], (uint32_t)__popc(loads) * 2u * Tr::kHalves * run_bytes);
+        }
+        __syncwarp();
+        if (load) {
+          const int y = (phys * Hkv + cur.kvh) * B + (u_t0 % B);
+          unsigned char* kt = smem + stage * Tr::kStageBytes + lane * unit_rows * 128;
+#pragma unroll
+          for (int hf = 0; hf < Tr::kHalves; ++hf) {
+            tma_load_2d(kt + hf * Tr::kSlabBytes, &prm.tmap_k, hf * 64, y, &full[stage], policy);
+            tma_load_2d(kt + Tr::kTileBytes + hf * Tr::kSlabBytes, &prm.tmap_v, hf * 64, y, &full[stage], policy);
+          }
+        }
+        if (i == 0 && !done) {
+          u_next = __shfl_sync(0xffffffffu, u_next_lane0, 0);
+          e_next = entry(u_next);
+        }
+      }
+      if (done || stop) break;
+      u = u_next;
+      cur = describe(u, e_next);
+    }
+    pdl_launch_dependents();
+    // never leave with copies in flight into this CTA's shared memory
+    if (lane == 0) {
+      int no_abort = 0;
+      for (int j = max(0, it - kTcStages); j < it; ++j)
+        if (!mbar_wait_bounded(&full[j % kTcStages], (j / kTcStages) & 1, &no_abort))
+          flag_error(PKV_DEV_WAIT_TIMEOUT);
+      if (nu > 0 && !mbar_wait_bounded(q_full, (nu - 1) & 1, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    // ----------------------------- MMA issuer -----------------------------
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = umma_idesc<T>(kTcRows, kTcTile, false);
+      constexpr uint32_t kIdescO = umma_idesc<T>(kTcRows, D, true);
+      const uint32_t q_base = smem_addr(smem + Tr::kQOffset);
+      const uint32_t p_hi = smem_addr(smem + Tr::kPOffset);
+      const uint32_t p_lo = p_hi + Tr::kPBytes;
+      bool ok = true;
+      int nu = 0;
+      // O += P V for the tile issued one step earlier
+      auto pv = [&](int it_prev, int stage_prev, bool first_prev) {
+        if (!mbar_wait_bounded(p_full, it_prev & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_addr(smem + stage_prev * Tr::kStageBytes + Tr::kTileBytes);
+#pragma unroll
+        for (int k = 0; k < kTcTile / 16; ++k) {
+          const uint64_t b = umma_desc_sw128(v_base + k * 16 * 128, Tr::kSlabBytes, 1024);
+          umma_f16(tmem_base + Tr::kOCol, umma_desc_sw128(p_hi + k * 32, 16, 1024), b, kIdescO,
+                   (first_prev && k == 0) ? 0u : 1u);
+          umma_f16(tmem_base + Tr::kOCol, umma_desc_sw128(p_lo + k * 32, 16, 1024), b, kIdescO, 1u);
+        }
+        umma_commit(&empty[stage_prev]);
+        umma_commit(o_done);
+        return true;
+      };
+      int it = 0;
+      bool have_prev = false;
+      int prev_stage = 0;
+      bool prev_first = false;
+      while (ok) {
+        const int stage = it % kTcStages;
+        if (!mbar_wait_bounded(&full[stage], (it / kTcStages) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int flags = hdr[2 * stage].w >> 16;
+        if (flags & kTileEnd) break;
+        const bool first = flags & kTileFirst;
+        if (first) {
+          if (!mbar_wait_bounded(q_full, nu & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ++nu;
+        }
+        const int sb = it & 1;
+        if (it >= 2 && !mbar_wait_bounded(&s_free[sb], ((it >> 1) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_base = smem_addr(smem + stage * Tr::kStageBytes);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (uint32_t)(k & 3) * 32u;  // 16 columns = 32 bytes inside a slab
+          const uint64_t a = umma_desc_sw128(q_base + (k >> 2) * Tr::kQSlabBytes + off, 16, 1024);
+          const uint64_t b = umma_desc_sw128(k_base + (k >> 2) * Tr::kSlabBytes + off, 16, 1024);
+          umma_f16(tmem_base + (uint32_t)(sb * kTcTile), a, b, kIdescS, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[sb]);
+        if (flags & kTileLast) umma_commit(q_empty);
+        if (have_prev && !pv(it - 1, prev_stage, prev_first)) {
+          ok = false;
+          break;
+        }
+        have_prev = true;
+        prev_stage = stage;
+        prev_first = first;
+        ++it;
+      }
+      if (ok && have_prev && !pv(it - 1, prev_stage, prev_first)) ok = false;
+      if (!ok) {
+        flag_error(PKV_DEV_WAIT_TIMEOUT);
+        *abort_flag = 1;
+      }
+      // every MMA issued above must be complete before the tensor memory is freed
+      umma_commit(drain);
+      int no_abort = 0;
+      if (!mbar_wait_bounded(drain, 0, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // --------------------------- softmax / epilogue ---------------------------
+    const int q4 = warp & 3;          // tensor-memory lane quarter of this warp
+    const int r = q4 * 32 + lane;     // query row of this thread
+    const uint32_t trow = tmem_base + ((uint32_t)(q4 * 32) << 16);
+    const int tq_local = r / G;
+    const bool row_in_tile = r < G * Tq;
+    float m_ref = -INFINITY, l = 0.f;
+    int4 uh = make_int4(0, 0, 0, 0);  // header of the unit being accumulated
+    bool have_unit = false;
+
+    // write this row of the finished unit: the final row, or the partition's state
+    auto finalize = [&]() {
+      const int us = uh.x, ukv = uh.y & 0xffff, urt = uh.y >> 16, up = uh.z & 0xffff, un = uh.z >> 16;
+      const int tq = urt * Tq + tq_local;
+      const bool real = row_in_tile && tq < prm.q_len;
+      const size_t sh = ((size_t)us * prm.q_len + tq) * prm.num_heads + (size_t)ukv * G + (r - tq_local * G);
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(trow + Tr::kOCol + 16 * c, v);
+        tmem_wait_ld16(v);
+        if (real) {
+          float4* dst = un == 1 ? reinterpret_cast<float4*>(prm.out + sh * D + 16 * c)
+                                : reinterpret_cast<float4*>(prm.ws_acc + (sh * prm.max_parts + up) * D + 16 * c);
+          const float f = un == 1 ? inv : 1.f;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            dst[k] = make_float4(__uint_as_float(v[4 * k]) * f, __uint_as_float(v[4 * k + 1]) * f,
+                                 __uint_as_float(v[4 * k + 2]) * f, __uint_as_float(v[4 * k + 3]) * f);
+        }
+      }
+      if (real && un != 1) prm.ws_ml[sh * prm.max_parts + up] = make_float2(m_ref, l);
+    };
+
+    bool failed = false;
+    for (int j = 0;; ++j) {
+      const int stage = j % kTcStages;
+      if (!mbar_wait_bounded(&full[stage], (j / kTcStages) & 1, abort_flag)) {
+        failed = true;
+        break;
+      }
+      const int4 hd = hdr[2 * stage];
+      const int4 hd2 = hdr[2 * stage + 1];
+      const int flags = hd.w >> 16;
+      const int n_valid = hd.w & 0xffff;
+      if (flags & kTileEnd) {
+        if (j >= 1) {
+          if (!mbar_wait_bounded(o_done, (j - 1) & 1, abort_flag)) {
+            failed = true;
+            break;
+          }
+          tc_fence_after();
+          if (have_unit) finalize();
+        }
+        break;
+      }
+      const int sb = j & 1;
+      if (!mbar_wait_bounded(&s_full[sb], (j >> 1) & 1, abort_flag)) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      float x[kTcTile];
+#pragma unroll
+      for (int c = 0; c < kTcTile / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(trow + (uint32_t)(sb * kTcTile + 16 * c), v);
+        tmem_wait_ld16(v);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[16 * c + k] = __uint_as_float(v[k]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[sb]);
+
+      // causal limit of this row: query token tq sees positions < ctx - Lq + tq + 1
+      const int t0 = hd2.x, ctx = hd2.y;
+      const int tq = (hd.y >> 16) * Tq + tq_local;
+      const int limit = (row_in_tile && tq < prm.q_len) ? ctx - prm.q_len + tq + 1 : 0;
+      const int n_ok = max(0, min(n_valid, limit - t0));  // columns [0, n_ok) are visible
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kTcTile; ++c) {
+        x[c] = c < n_ok ? x[c] * prm.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, x[c]);
+      }
+
+      // PV of the previous tile is complete: O is stable and the P buffer is free
+      if (j >= 1 && !mbar_wait_bounded(o_done, (j - 1) & 1, abort_flag)) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      const bool first = flags & kTileFirst;
+      if (first) {
+        if (have_unit) finalize();
+        uh = hd;
+        have_unit = true;
+        m_ref = mt;
+        l = 0.f;
+      } else {
+        const bool need = mt > m_ref + kTcRescaleLog2;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? exp2f(m_ref - mt) : 1.f;  // 0 while m_ref is -inf
+          if (need) {
+            l *= alpha;
+            m_ref = mt;
+          }
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t v[16];
+            tmem_ld16(trow + Tr::kOCol + 16 * c, v);
+            tmem_wait_ld16(v);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
+            tmem_st16(trow + Tr::kOCol + 16 * c, v);
+          }
+          tmem_wait_st();
+        }
+      }
+
+      // P = 2^(x - m_ref) as high + low 16-bit parts, row r of the 128B-swizzled slab
+      unsigned char* phi = smem + Tr::kPOffset + r * 128;
+      unsigned char* plo = phi + Tr::kPBytes;
+#pragma unroll
+      for (int ch = 0; ch < kTcTile / 8; ++ch) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int c = 8 * ch + 2 * k;
+          const float p0 = x[c] == -INFINITY ? 0.f : exp2f(x[c] - m_ref);
+          const float p1 = x[c + 1] == -INFINITY ? 0.f : exp2f(x[c + 1] - m_ref);
+          l += p0 + p1;
+          const float h0 = round16<T>(p0), h1 = round16<T>(p1);
+          hi[k] = Mma16816<T>::pack(h0, h1);
+          lo[k] = Mma16816<T>::pack(p0 - h0, p1 - h1);
+        }
+        const int sw = (ch ^ (r & 7)) << 4;
+        *reinterpret_cast<uint4*>(phi + sw) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(plo + sw) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      // V rows past the tile's valid tokens may hold anything (NaN in unwritten
+      // slots): zero them so that 0 * V stays 0
+      if (n_valid < kTcTile) {
+        unsigned char* vt = smem + stage * Tr::kStageBytes + Tr::kTileBytes;
+        const int chunks = (kTcTile - n_valid) * 8 * Tr::kHalves;
+        for (int i = (warp - 2) * 32 + lane; i < chunks; i += 128) {
+          const int hf = i / ((kTcTile - n_valid) * 8);
+          const int rem = i - hf * (kTcTile - n_valid) * 8;
+          *reinterpret_cast<uint4*>(vt + hf * Tr::kSlabBytes + (n_valid + rem / 8) * 128 + (rem % 8) * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async_smem();  // P and the zeroed rows are read by the tensor cores
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (failed && lane == 0) {
+      flag_error(PKV_DEV_WAIT_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+
+  // free the tensor memory once every role is done with it
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTcTmemCols)
+                 : "memory");
+  }
+}
+
+}  // namespace pkv

@@ -16,6 +16,7 @@
 #include "pkv_device.cuh"
 #include "decode.cuh"
 #include "decode_gqa.cuh"
+#include "multi_query_tc.cuh"
 #include "cache_ops.cuh"
 
 namespace {
@@ -282,6 +283,22 @@ bool use_gqa_kernel(int Hq, int Hkv, int B, int NB, pkv_dtype dt) {
   return G >= 2 && G <= pkv::kGqaRows && dt != PKV_F32 && (long long)NB * Hkv * B < (1LL << 31);
 }
 
+// More than 16 query rows per K/V head (Lq * G) run on the tcgen05 kernel with
+// 128-row tiles of floor(128 / G) whole query tokens; up to 16 rows on the
+// mma.sync kernel's 16-row tiles.  The choice depends only on the shapes, so the
+// workspace query and the launch agree.
+bool mq_uses_tcgen05(long long q_len, int group, int head_dim) {
+  return q_len * group > pkv::kGqaRows && group <= pkv::kTcRows && (head_dim == 64 || head_dim == 128);
+}
+
+long long mq_row_tiles(long long q_len, int group, int head_dim) {
+  if (mq_uses_tcgen05(q_len, group, head_dim)) {
+    const long long tq = pkv::kTcRows / group;
+    return (q_len + tq - 1) / tq;
+  }
+  return (q_len * group + pkv::kGqaRows - 1) / pkv::kGqaRows;
+}
+
 // Launch the tensor-core kernel for Lq query tokens per sequence over the plan's
 // unit list (the plan kernel has been launched already).
 int launch_tensor_core(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
@@ -321,6 +338,96 @@ int launch_tensor_core(const void* q, const void* k_cache, const void* v_cache, 
     return head_dim == 64 ? launch_gqa<__nv_bfloat16, 64, 3>(g, max_units, st)
                           : launch_gqa<__nv_bfloat16, 128, 3>(g, max_units, st);
   return head_dim == 64 ? launch_gqa<__half, 64, 3>(g, max_units, st) : launch_gqa<__half, 128, 3>(g, max_units, st);
+}
+
+// 4-D view [S][Lq][Hq][D] of the query rows (16-bit); boxes of 64 columns x G heads
+// x Tq tokens x 1 sequence, 128-byte swizzle, so that one box lands as the
+// 128-byte-swizzled rows r = token * G + head of a 128-row operand tile.
+int encode_query_map(CUtensorMap* map, const void* q, int S, int Lq, int Hq, int D, int G, int Tq, pkv_dtype dt) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  if (tensor_map_encoder(&enc) != PKV_OK) return PKV_ECUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)Lq, (cuuint64_t)S};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2, (cuuint64_t)Lq * Hq * D * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)Tq, 1};
+  const cuuint32_t elem_strides[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType type =
+      dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUresult r = enc(map, type, 4, const_cast<void*>(q), dims, strides, box, elem_strides,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ECUDA;
+}
+
+template <typename T, int D>
+int launch_tc(const pkv::TcParams& prm, long long max_units, cudaStream_t st) {
+  using Tr = pkv::TcTraits<D>;
+  static bool attr_set[kMaxDevices];
+  int dev;
+  if (current_device(&dev) != PKV_OK) return PKV_ECUDA;
+  const int sms = sm_count(dev);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(pkv::paged_multi_query_tc_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Tr::kSmemAlloc) != cudaSuccess)
+        return PKV_ECUDA;
+      attr_set[dev] = true;
+    }
+  }
+  if (sms <= 0) return PKV_ECUDA;
+  long long grid = sms;  // one CTA per SM (shared memory and tensor memory)
+  if (grid > max_units) grid = max_units;
+  if (grid < 1) grid = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(pkv::kTcThreads);
+  cfg.dynamicSmemBytes = Tr::kSmemAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, pkv::paged_multi_query_tc_kernel<T, D>, prm) != cudaSuccess) return PKV_ECUDA;
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+int launch_tcgen05(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables, int num_seqs,
+                   int q_len, int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                   int num_blocks, pkv_dtype dtype, float scale_log2, float* out, const DecodePlan& plan,
+                   const pkv::DecodeParams& prm, cudaStream_t st) {
+  static_assert(alignof(pkv::TcParams) >= 64, "tensor maps need 64-byte alignment");
+  pkv::TcParams t;
+  const int G = num_heads / num_kv_heads;
+  const int Tq = pkv::kTcRows / G;
+  const long long rows = (long long)num_blocks * num_kv_heads * block_size;
+  const int box_rows = block_size < pkv::kTcTile ? block_size : pkv::kTcTile;
+  if (encode_pool_map(&t.tmap_k, k_cache, rows, head_dim, box_rows, dtype) != PKV_OK ||
+      encode_pool_map(&t.tmap_v, v_cache, rows, head_dim, box_rows, dtype) != PKV_OK ||
+      encode_query_map(&t.tmap_q, q, num_seqs, q_len, num_heads, head_dim, G, Tq, dtype) != PKV_OK)
+    return PKV_ECUDA;
+  t.block_tables = block_tables;
+  t.num_heads = num_heads;
+  t.num_kv_heads = num_kv_heads;
+  t.group = G;
+  t.q_len = q_len;
+  t.tq_per_tile = Tq;
+  t.row_tiles = (int)mq_row_tiles(q_len, G, head_dim);
+  t.block_size = block_size;
+  t.max_blocks = max_blocks_per_seq;
+  t.num_blocks = num_blocks;
+  t.scale_log2 = scale_log2;
+  t.part_tokens = plan.part_tokens;
+  t.max_parts = plan.max_parts;
+  t.out = out;
+  t.ws_acc = prm.ws_acc;
+  t.ws_ml = prm.ws_ml;
+  t.units = prm.units;
+  t.counters = prm.counters;
+  const long long max_units = (long long)num_seqs * num_kv_heads * t.row_tiles * plan.max_parts;
+  if (dtype == PKV_BF16)
+    return head_dim == 64 ? launch_tc<__nv_bfloat16, 64>(t, max_units, st) : launch_tc<__nv_bfloat16, 128>(t, max_units, st);
+  return head_dim == 64 ? launch_tc<__half, 64>(t, max_units, st) : launch_tc<__half, 128>(t, max_units, st);
 }
 
 // The merge is a programmatic dependent of the decode kernel: its CTAs may be
@@ -454,12 +561,11 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const i
   return result;
 }
 
-// Several query tokens per sequence (tensor-core kernel only: 16-bit K/V).
+// Several query tokens per sequence (tensor-core kernels only: 16-bit K/V).
 int multi_query_plan(int num_seqs, int q_len, int num_heads, int num_kv_heads, int head_dim, int block_size,
                      int max_blocks_per_seq, int partition_tokens, DecodePlan* plan) {
   if (q_len <= 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0) return PKV_EINVAL;
-  const long long rows = (long long)q_len * (num_heads / num_kv_heads);
-  const long long row_tiles = (rows + pkv::kGqaRows - 1) / pkv::kGqaRows;
+  const long long row_tiles = mq_row_tiles(q_len, num_heads / num_kv_heads, head_dim);
   if (row_tiles > 32767 || (long long)q_len * num_heads > 65535) return PKV_EINVAL;
   return make_plan(num_seqs, q_len * num_heads, (int)(num_kv_heads * row_tiles), head_dim, block_size,
                    max_blocks_per_seq, partition_tokens, plan);
@@ -505,7 +611,11 @@ int multi_query_impl(const void* q, const void* k_cache, const void* v_cache, co
       context_lens, num_seqs, max_ctx, plan.part_tokens, plan.sort ? 1 : 0,
       reinterpret_cast<uint2*>(ws + plan.off_units), prm.counters);
   if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
-  if (result == PKV_OK)
+  if (result == PKV_OK && mq_uses_tcgen05(q_len, num_heads / num_kv_heads, head_dim))
+    result = launch_tcgen05(q, k_cache, v_cache, block_tables, num_seqs, q_len, num_heads, num_kv_heads, head_dim,
+                            block_size, max_blocks_per_seq, num_blocks, dtype, scale * pkv::kLog2e, out, plan, prm,
+                            st);
+  else if (result == PKV_OK)
     result = launch_tensor_core(q, k_cache, v_cache, block_tables, context_lens, num_seqs, q_len, num_heads,
                                 num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, dtype,
                                 scale * pkv::kLog2e, out, plan, prm, st);
