@@ -60,7 +60,7 @@ def parse():
                     help="query tokens per sequence (>1: verify / chunked-prefill step through "
                          "paged_attn_multi_query; the last q_len positions are appended each step)")
     ap.add_argument("--num-seqs", type=int, default=None,
-                    help="profiling aid: fewer sequences of the opt13b layer (a smaller case for ncu)")
+                    help="profiling aid: fewer sequences of the opt13b or gqa layers (a smaller case for ncu)")
     a = ap.parse_args()
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
@@ -294,6 +294,9 @@ def run_gpu(a, rank, world, local_rank):
 
     if a.num_seqs is not None and a.workload == "opt13b":
         w = wl.make_opt13b(B=a.block_size, device=dev, S=a.num_seqs)
+        w.name += f"_S{a.num_seqs}"
+    elif a.num_seqs is not None and a.workload.startswith("gqa"):
+        w = wl.make_gqa(int(a.workload[3:]), device=dev, S=a.num_seqs, B=a.block_size)
         w.name += f"_S{a.num_seqs}"
     else:
         w = wl.make(a.workload, device=dev, B=a.block_size if a.workload in ("opt13b",) or

@@ -15,7 +15,9 @@
 //   P = 2^(S*scale - m) four softmax warps, one row per thread, S read from tensor memory
 //   O += P V            tcgen05.mma  M=128 N=D   K=64  (P from shared memory, V as an MN-major operand)
 //
-// S (double-buffered, 2 x 64 columns) and O (D columns) live in tensor memory.
+// S (double-buffered, 2 x 64 columns) and O (D columns) live in tensor memory; P
+// is double-buffered in shared memory, so the softmax of tile j+1 overlaps the
+// P V product of tile j.
 // P is split into a 16-bit high part and the 16-bit rounding of the rest, and both
 // are multiplied (with P rounded to 16 bits alone the error exceeds 2e-3).  O is
 // rescaled only when a row's running maximum grows by more than 2^8 (the partial
@@ -38,7 +40,7 @@ namespace pkv {
 
 constexpr int kTcRows = 128;          // M: query rows per tile = tensor-memory lanes
 constexpr int kTcTile = 64;           // tokens per K/V tile
-constexpr int kTcStages = 3;
+constexpr int kTcStages = 4;  // the P V product of tile t is issued after S of tile t + 2
 constexpr int kTcThreads = 6 * 32;    // producer, MMA, four softmax warps
 constexpr int kTcTmemCols = 256;      // S[2] at columns 0 and 64, O at column 128
 constexpr float kTcRescaleLog2 = 8.0f;
@@ -76,11 +78,11 @@ struct TcTraits {
   static constexpr int kQSlabBytes = kTcRows * 128;         // 128 rows x 64 columns
   static constexpr int kQOffset = kTcStages * kStageBytes;
   static constexpr int kPBytes = kTcRows * kTcTile * 2;     // 128 rows x 64 tokens, one slab
-  static constexpr int kPOffset = kQOffset + kHalves * kQSlabBytes;  // P high, then P low
-  static constexpr int kHdrOffset = kPOffset + 2 * kPBytes;          // two int4 per stage
+  static constexpr int kPOffset = kQOffset + kHalves * kQSlabBytes;  // [2 buffers][P high, P low]
+  static constexpr int kHdrOffset = kPOffset + 4 * kPBytes;          // two int4 per stage
   static constexpr int kBarOffset = kHdrOffset + kTcStages * 32;
-  // full[NS], empty[NS], q_full, q_empty, s_full[2], s_free[2], p_full, o_done, drain
-  static constexpr int kNumBars = 2 * kTcStages + 9;
+  // full[NS], empty[NS], q_full, q_empty, s_full[2], s_free[2], p_full[2], o_done[2], drain
+  static constexpr int kNumBars = 2 * kTcStages + 11;
   static constexpr int kTmemSlotOffset = kBarOffset + kNumBars * 8;
   static constexpr int kAbortOffset = kTmemSlotOffset + 8;
   static constexpr int kSmemBytes = kAbortOffset + 8;
@@ -159,6 +161,31 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// 32 consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Redefine 32 registers after a tcgen05.wait::ld so that no use is scheduled above it.
+__device__ __forceinline__ void tmem_pin32(uint32_t* r) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 // Wait for this thread's tensor-memory loads, then pin the loaded registers after
 // the wait (the empty asm redefines them, so no use is scheduled above it).
 __device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
@@ -180,15 +207,23 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// (p0, p1) -> high parts (p in T) and low parts (T rounding of p - high), each as a
+// packed pair; high + low carries ~16 more bits of p than high alone.
 template <typename T>
-__device__ __forceinline__ float round16(float a);
+__device__ __forceinline__ void split_pair(float p0, float p1, uint32_t& hi, uint32_t& lo);
 template <>
-__device__ __forceinline__ float round16<__half>(float a) {
-  return __half2float(__float2half_rn(a));
+__device__ __forceinline__ void split_pair<__nv_bfloat16>(float p0, float p1, uint32_t& hi, uint32_t& lo) {
+  hi = Mma16816<__nv_bfloat16>::pack(p0, p1);
+  // a bf16 is the top half of an fp32
+  lo = Mma16816<__nv_bfloat16>::pack(p0 - __uint_as_float(hi << 16), p1 - __uint_as_float(hi & 0xffff0000u));
 }
 template <>
-__device__ __forceinline__ float round16<__nv_bfloat16>(float a) {
-  return __bfloat162float(__float2bfloat16_rn(a));
+__device__ __forceinline__ void split_pair<__half>(float p0, float p1, uint32_t& hi, uint32_t& lo) {
+  hi = Mma16816<__half>::pack(p0, p1);
+  __half2 h;
+  memcpy(&h, &hi, 4);
+  const float2 f = __half22float2(h);
+  lo = Mma16816<__half>::pack(p0 - f.x, p1 - f.y);
 }
 
 struct TcUnit {
@@ -208,9 +243,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
   uint64_t* q_empty = q_full + 1;
   uint64_t* s_full = q_full + 2;  // [2]
   uint64_t* s_free = q_full + 4;  // [2]
-  uint64_t* p_full = q_full + 6;
-  uint64_t* o_done = q_full + 7;
-  uint64_t* drain = q_full + 8;
+  uint64_t* p_full = q_full + 6;  // [2]: P buffer b of tile j = j & 1 written
+  uint64_t* o_done = q_full + 8;  // [2]: P V of tile j (j & 1 = b) complete
+  uint64_t* drain = q_full + 10;
   int4* hdr = reinterpret_cast<int4*>(smem + Tr::kHdrOffset);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::kTmemSlotOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Tr::kAbortOffset);
@@ -235,8 +270,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
     mbar_init(&s_full[1], 1);
     mbar_init(&s_free[0], 4);
     mbar_init(&s_free[1], 4);
-    mbar_init(p_full, 4);
-    mbar_init(o_done, 1);
+    mbar_init(&p_full[0], 4);
+    mbar_init(&p_full[1], 4);
+    mbar_init(&o_done[0], 1);
+    mbar_init(&o_done[1], 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -393,14 +430,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
       constexpr uint32_t kIdescS = umma_idesc<T>(kTcRows, kTcTile, false);
       constexpr uint32_t kIdescO = umma_idesc<T>(kTcRows, D, true);
       const uint32_t q_base = smem_addr(smem + Tr::kQOffset);
-      const uint32_t p_hi = smem_addr(smem + Tr::kPOffset);
-      const uint32_t p_lo = p_hi + Tr::kPBytes;
+      const uint32_t p_base = smem_addr(smem + Tr::kPOffset);
       bool ok = true;
       int nu = 0;
       // O += P V for the tile issued one step earlier
       auto pv = [&](int it_prev, int stage_prev, bool first_prev) {
-        if (!mbar_wait_bounded(p_full, it_prev & 1, abort_flag)) return false;
+        const int pb = it_prev & 1;
+        if (!mbar_wait_bounded(&p_full[pb], (it_prev >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
+        const uint32_t p_hi = p_base + pb * 2 * Tr::kPBytes;
+        const uint32_t p_lo = p_hi + Tr::kPBytes;
         const uint32_t v_base = smem_addr(smem + stage_prev * Tr::kStageBytes + Tr::kTileBytes);
 #pragma unroll
         for (int k = 0; k < kTcTile / 16; ++k) {
@@ -410,13 +449,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
           umma_f16(tmem_base + Tr::kOCol, umma_desc_sw128(p_lo + k * 32, 16, 1024), b, kIdescO, 1u);
         }
         umma_commit(&empty[stage_prev]);
-        umma_commit(o_done);
+        umma_commit(&o_done[pb]);
         return true;
       };
+      // S of tile t is issued as soon as its K/V and S buffer are ready; the P V
+      // product of tile t - 2 follows it (of tile t - 1 too when tile t opens a new
+      // unit, whose epilogue reads O), so the tensor pipe always holds an S product
+      // ahead of the softmax warps.
       int it = 0;
-      bool have_prev = false;
-      int prev_stage = 0;
-      bool prev_first = false;
+      int pv_next = 0;               // first tile whose P V product is not issued
+      bool first_of[2] = {false, false};  // first-tile flags of the tiles in flight, by t & 1
+      auto pv_upto = [&](int t_last) {
+        while (ok && pv_next <= t_last) {
+          const bool f = (pv_next & 1) ? first_of[1] : first_of[0];
+          if (!pv(pv_next, pv_next % kTcStages, f)) ok = false;
+          ++pv_next;
+        }
+      };
       while (ok) {
         const int stage = it % kTcStages;
         if (!mbar_wait_bounded(&full[stage], (it / kTcStages) & 1, abort_flag)) {
@@ -449,16 +498,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
         }
         umma_commit(&s_full[sb]);
         if (flags & kTileLast) umma_commit(q_empty);
-        if (have_prev && !pv(it - 1, prev_stage, prev_first)) {
-          ok = false;
-          break;
-        }
-        have_prev = true;
-        prev_stage = stage;
-        prev_first = first;
+        // tiles t - 2 and t share a history slot: issue the pending products first
+        pv_upto(first ? it - 1 : it - 2);
+        if (sb)
+          first_of[1] = first;
+        else
+          first_of[0] = first;
         ++it;
       }
-      if (ok && have_prev && !pv(it - 1, prev_stage, prev_first)) ok = false;
+      if (ok) pv_upto(it - 1);
       if (!ok) {
         flag_error(PKV_DEV_WAIT_TIMEOUT);
         *abort_flag = 1;
@@ -479,6 +527,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
     float m_ref = -INFINITY, l = 0.f;
     int4 uh = make_int4(0, 0, 0, 0);  // header of the unit being accumulated
     bool have_unit = false;
+    bool failed = false;
+    // P V products confirmed complete, per P buffer (each o_done phase is waited in order)
+    int pv_seen0 = 0, pv_seen1 = 0;
+    auto wait_pv = [&](int t) {  // P V of tile t (t >= 0) complete
+      const int b = t & 1, k = t >> 1;
+      int& seen = b ? pv_seen1 : pv_seen0;
+      if (k < seen) return true;
+      if (!mbar_wait_bounded(&o_done[b], k & 1, abort_flag)) return false;
+      seen = k + 1;
+      return true;
+    };
 
     // write this row of the finished unit: the final row, or the partition's state
     auto finalize = [&]() {
@@ -486,18 +545,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
       const int tq = urt * Tq + tq_local;
       const bool real = row_in_tile && tq < prm.q_len;
       const size_t sh = ((size_t)us * prm.q_len + tq) * prm.num_heads + (size_t)ukv * G + (r - tq_local * G);
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const float f = un == 1 ? ((l > 0.f) ? 1.f / l : 0.f) : 1.f;
+      float* dst_row = un == 1 ? prm.out + sh * D : prm.ws_acc + (sh * prm.max_parts + up) * D;
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld16(trow + Tr::kOCol + 16 * c, v);
-        tmem_wait_ld16(v);
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(trow + Tr::kOCol + 32 * c, v);
+        tmem_wait_ld();
+        tmem_pin32(v);
         if (real) {
-          float4* dst = un == 1 ? reinterpret_cast<float4*>(prm.out + sh * D + 16 * c)
-                                : reinterpret_cast<float4*>(prm.ws_acc + (sh * prm.max_parts + up) * D + 16 * c);
-          const float f = un == 1 ? inv : 1.f;
+          float4* dst = reinterpret_cast<float4*>(dst_row + 32 * c);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
+          for (int k = 0; k < 8; ++k)
             dst[k] = make_float4(__uint_as_float(v[4 * k]) * f, __uint_as_float(v[4 * k + 1]) * f,
                                  __uint_as_float(v[4 * k + 2]) * f, __uint_as_float(v[4 * k + 3]) * f);
         }
@@ -505,7 +564,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
       if (real && un != 1) prm.ws_ml[sh * prm.max_parts + up] = make_float2(m_ref, l);
     };
 
-    bool failed = false;
     for (int j = 0;; ++j) {
       const int stage = j % kTcStages;
       if (!mbar_wait_bounded(&full[stage], (j / kTcStages) & 1, abort_flag)) {
@@ -517,14 +575,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
       const int flags = hd.w >> 16;
       const int n_valid = hd.w & 0xffff;
       if (flags & kTileEnd) {
-        if (j >= 1) {
-          if (!mbar_wait_bounded(o_done, (j - 1) & 1, abort_flag)) {
-            failed = true;
-            break;
-          }
-          tc_fence_after();
-          if (have_unit) finalize();
+        // the last unit's products must be complete before its rows are read
+        if ((j >= 2 && !wait_pv(j - 2)) || (j >= 1 && !wait_pv(j - 1))) {
+          failed = true;
+          break;
         }
+        tc_fence_after();
+        if (have_unit) finalize();
         break;
       }
       const int sb = j & 1;
@@ -534,13 +591,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
       }
       tc_fence_after();
       float x[kTcTile];
+      {
+        uint32_t v[kTcTile];
+        tmem_ld32(trow + (uint32_t)(sb * kTcTile), v);
+        tmem_ld32(trow + (uint32_t)(sb * kTcTile + 32), v + 32);
+        tmem_wait_ld();
+        tmem_pin32(v);
+        tmem_pin32(v + 32);
 #pragma unroll
-      for (int c = 0; c < kTcTile / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld16(trow + (uint32_t)(sb * kTcTile + 16 * c), v);
-        tmem_wait_ld16(v);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) x[16 * c + k] = __uint_as_float(v[k]);
+        for (int c = 0; c < kTcTile; ++c) x[c] = __uint_as_float(v[c]);
       }
       tc_fence_before();
       __syncwarp();
@@ -558,23 +617,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
         mt = fmaxf(mt, x[c]);
       }
 
-      // PV of the previous tile is complete: O is stable and the P buffer is free
-      if (j >= 1 && !mbar_wait_bounded(o_done, (j - 1) & 1, abort_flag)) {
+      // P buffer j & 1 was last read by the P V product of tile j - 2
+      if (j >= 2 && !wait_pv(j - 2)) {
         failed = true;
         break;
       }
-      tc_fence_after();
       const bool first = flags & kTileFirst;
-      if (first) {
-        if (have_unit) finalize();
-        uh = hd;
-        have_unit = true;
-        m_ref = mt;
-        l = 0.f;
-      } else {
-        const bool need = mt > m_ref + kTcRescaleLog2;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? exp2f(m_ref - mt) : 1.f;  // 0 while m_ref is -inf
+      const bool need = !first && mt > m_ref + kTcRescaleLog2;
+      // O is touched (read for the previous unit's rows, or rescaled): every product so far must be done
+      if ((first && have_unit) || __any_sync(0xffffffffu, need)) {
+        if (j >= 1 && !wait_pv(j - 1)) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+        if (first) {
+          finalize();
+        } else {
+          const float alpha = need ? ex2_fast(m_ref - mt) : 1.f;  // 0 while m_ref is -inf
           if (need) {
             l *= alpha;
             m_ref = mt;
@@ -591,9 +651,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
           tmem_wait_st();
         }
       }
+      if (first) {
+        uh = hd;
+        have_unit = true;
+        m_ref = mt;
+        l = 0.f;
+      }
 
       // P = 2^(x - m_ref) as high + low 16-bit parts, row r of the 128B-swizzled slab
-      unsigned char* phi = smem + Tr::kPOffset + r * 128;
+      unsigned char* phi = smem + Tr::kPOffset + sb * 2 * Tr::kPBytes + r * 128;
       unsigned char* plo = phi + Tr::kPBytes;
 #pragma unroll
       for (int ch = 0; ch < kTcTile / 8; ++ch) {
@@ -601,12 +667,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int c = 8 * ch + 2 * k;
-          const float p0 = x[c] == -INFINITY ? 0.f : exp2f(x[c] - m_ref);
-          const float p1 = x[c + 1] == -INFINITY ? 0.f : exp2f(x[c + 1] - m_ref);
+          const float p0 = x[c] == -INFINITY ? 0.f : ex2_fast(x[c] - m_ref);
+          const float p1 = x[c + 1] == -INFINITY ? 0.f : ex2_fast(x[c + 1] - m_ref);
           l += p0 + p1;
-          const float h0 = round16<T>(p0), h1 = round16<T>(p1);
-          hi[k] = Mma16816<T>::pack(h0, h1);
-          lo[k] = Mma16816<T>::pack(p0 - h0, p1 - h1);
+          split_pair<T>(p0, p1, hi[k], lo[k]);
         }
         const int sw = (ch ^ (r & 7)) << 4;
         *reinterpret_cast<uint4*>(phi + sw) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -627,7 +691,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
       fence_proxy_async_smem();  // P and the zeroed rows are read by the tensor cores
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[sb]);
     }
     if (failed && lane == 0) {
       flag_error(PKV_DEV_WAIT_TIMEOUT);
