@@ -37,9 +37,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention effective KV GB/s and % of B200 HBM peak"
 FALLBACK_HBM_GBS = 6650.0
-WORKLOADS = ("opt13b", "llama7b", "cow", "longctx", "tiny", "gqa2", "gqa4", "gqa8", "gqa16", "swap")
+WORKLOADS = ("opt13b", "llama7b", "cow", "longctx", "tiny", "gqa2", "gqa4", "gqa8", "gqa16", "gqa32", "gqa64", "swap")
 DEFAULT_STEPS = {"opt13b": 500, "llama7b": 2000, "cow": 1000, "longctx": 500, "tiny": 200,
-                 "gqa2": 500, "gqa4": 500, "gqa8": 500, "gqa16": 500, "swap": 20}
+                 "gqa2": 500, "gqa4": 500, "gqa8": 500, "gqa16": 500, "gqa32": 300, "gqa64": 300, "swap": 20}
 
 
 def parse():

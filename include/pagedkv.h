@@ -158,6 +158,10 @@ int paged_attn_decode_partition_tokens(int num_seqs, int num_heads, int head_dim
  *   Every other argument, the return codes and the device-side checks are those of
  *   paged_attn_decode; num_kv_heads == num_heads is exactly paged_attn_decode.
  *   The workspace size comes from paged_attn_decode_gqa_workspace_size.
+ *
+ * With 16-bit K/V, 2 <= G <= 16 query heads per K/V head run on a warp-level
+ * tensor-core kernel (16-row tiles) and 16 < G <= 128 on a tcgen05 kernel (one
+ * 128-row tile per (sequence, K/V head)); fp32 K/V and other G on CUDA cores.
  */
 int paged_attn_decode_gqa(const void* q, const void* k_cache, const void* v_cache,
                           const int32_t* block_tables, const int32_t* context_lens,
@@ -223,6 +227,10 @@ size_t paged_attn_decode_tune_workspace_size(int num_seqs, int num_heads, int nu
  *   out           float32 [num_seqs][q_len][num_heads][head_dim].
  *   The rest is as in paged_attn_decode_gqa; fp32 storage returns PKV_EUNSUPPORTED.
  *   q_len = 1 computes exactly what paged_attn_decode_gqa computes.
+ *
+ * R = q_len * G query rows per (sequence, K/V head): R <= 16 runs on the warp-level
+ * tensor-core kernel; R > 16 (with G <= 128 and head_dim 64 or 128) on the tcgen05
+ * kernel, 128-row tiles of floor(128 / G) query tokens, K/V read once per tile.
  */
 int paged_attn_multi_query(const void* q, const void* k_cache, const void* v_cache,
                            const int32_t* block_tables, const int32_t* context_lens,

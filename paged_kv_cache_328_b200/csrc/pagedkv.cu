@@ -547,6 +547,11 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const i
     result = launch_tensor_core(q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1, num_heads,
                                 num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, dtype, prm.scale_log2,
                                 out, plan, prm, st);
+  } else if (result == PKV_OK && dtype != PKV_F32 && mq_uses_tcgen05(1, num_heads / num_kv_heads, head_dim) &&
+             (long long)num_blocks * num_kv_heads * block_size < (1LL << 31)) {
+    // more than 16 query heads per K/V head: one 128-row tcgen05 tile per (sequence, K/V head)
+    result = launch_tcgen05(q, k_cache, v_cache, block_tables, num_seqs, 1, num_heads, num_kv_heads, head_dim,
+                            block_size, max_blocks_per_seq, num_blocks, dtype, prm.scale_log2, out, plan, prm, st);
   } else if (result == PKV_OK) {
     const long long max_units = (long long)num_seqs * num_heads * plan.max_parts;
     result = head_dim == 64 ? dispatch_decode<64>(dtype, prm, max_units, st)

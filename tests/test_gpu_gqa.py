@@ -1,7 +1,8 @@
 """GPU parity of grouped-query paged decode (paged_attn_decode_gqa through the C ABI).
 
 Query head h reads K/V head h // G.  16-bit K/V with 2 <= G <= 16 runs on the
-tensor-core kernel; fp32 K/V, G = 1 and G > 16 run on the CUDA-core kernel.
+warp-level tensor-core kernel, 16 < G <= 128 on the tcgen05 kernel (one 128-row
+tile per (sequence, K/V head)); fp32 K/V and G = 1 run on the CUDA-core kernel.
 Tolerances as for multi-head decode: 2e-3 (fp16/bf16), 1e-5 (fp32).
 """
 
@@ -37,7 +38,7 @@ def full_oracle(w):
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
-@pytest.mark.parametrize("G", [2, 3, 4, 7, 8, 16, 32])
+@pytest.mark.parametrize("G", [2, 3, 4, 7, 8, 16, 32, 48, 128])
 @pytest.mark.parametrize("D", [64, 128])
 def test_gqa_small_ragged(dev, dtype, G, D):
     Hkv = 2
