@@ -13,11 +13,13 @@
 //
 //   S = Q K^T           tcgen05.mma  M=128 N=64  K=D   (Q and the K tile from shared memory)
 //   P = 2^(S*scale - m) four softmax warps, one row per thread, S read from tensor memory
-//   O += P V            tcgen05.mma  M=128 N=D   K=64  (P from shared memory, V as an MN-major operand)
+//   O += P V            tcgen05.mma  M=128 N=D   K=64  (P from tensor memory, V as an MN-major operand)
 //
-// S (double-buffered, 2 x 64 columns) and O (D columns) live in tensor memory; P
-// is double-buffered in shared memory, so the softmax of tile j+1 overlaps the
-// P V product of tile j.
+// S (double-buffered, 2 x 64 columns), O (D columns) and P (double-buffered, 2 x
+// 64 columns of packed 16-bit pairs) live in tensor memory: the softmax threads
+// store P with tcgen05.st into their own lanes and the P V product reads it as its
+// A operand, so P never touches shared memory, and the softmax of tile j+1
+// overlaps the P V product of tile j.
 // P is split into a 16-bit high part and the 16-bit rounding of the rest, and both
 // are multiplied (with P rounded to 16 bits alone the error exceeds 2e-3).  O is
 // rescaled only when a row's running maximum grows by more than 2^8 (the partial
@@ -40,9 +42,9 @@ namespace pkv {
 
 constexpr int kTcRows = 128;          // M: query rows per tile = tensor-memory lanes
 constexpr int kTcTile = 64;           // tokens per K/V tile
-constexpr int kTcStages = 4;  // the P V product of tile t is issued after S of tile t + 2
+constexpr int kTcStages = 6;  // the P V product of tile t is issued after S of tile t + 2
 constexpr int kTcThreads = 6 * 32;    // producer, MMA, four softmax warps
-constexpr int kTcTmemCols = 256;      // S[2] at columns 0 and 64, O at column 128
+constexpr int kTcTmemCols = 512;      // S[2] at columns 0 and 64, O at 128, P[2] (high, low) at 256 and 320
 constexpr float kTcRescaleLog2 = 8.0f;
 
 struct TcParams {
@@ -77,9 +79,7 @@ struct TcTraits {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kQSlabBytes = kTcRows * 128;         // 128 rows x 64 columns
   static constexpr int kQOffset = kTcStages * kStageBytes;
-  static constexpr int kPBytes = kTcRows * kTcTile * 2;     // 128 rows x 64 tokens, one slab
-  static constexpr int kPOffset = kQOffset + kHalves * kQSlabBytes;  // [2 buffers][P high, P low]
-  static constexpr int kHdrOffset = kPOffset + 4 * kPBytes;          // two int4 per stage
+  static constexpr int kHdrOffset = kQOffset + kHalves * kQSlabBytes;  // two int4 per stage
   static constexpr int kBarOffset = kHdrOffset + kTcStages * 32;
   // full[NS], empty[NS], q_full, q_empty, s_full[2], s_free[2], p_full[2], o_done[2], drain
   static constexpr int kNumBars = 2 * kTcStages + 11;
@@ -88,8 +88,9 @@ struct TcTraits {
   static constexpr int kSmemBytes = kAbortOffset + 8;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;      // the base is rounded up to 1024 bytes
   static constexpr uint32_t kOCol = 128;
+  static constexpr uint32_t kPCol = 256;  // P buffer b: high part at kPCol + 64 b, low part 32 columns on
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
-  static_assert(kQOffset % 1024 == 0 && kPOffset % 1024 == 0, "swizzle atoms are 1024-byte aligned");
+  static_assert(kQOffset % 1024 == 0, "swizzle atoms are 1024-byte aligned");
   static_assert(kSmemAlloc <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -129,6 +130,17 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same with the A operand (K-major, 16-bit pairs per 32-bit column) in tensor memory.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -430,7 +442,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
       constexpr uint32_t kIdescS = umma_idesc<T>(kTcRows, kTcTile, false);
       constexpr uint32_t kIdescO = umma_idesc<T>(kTcRows, D, true);
       const uint32_t q_base = smem_addr(smem + Tr::kQOffset);
-      const uint32_t p_base = smem_addr(smem + Tr::kPOffset);
+
       bool ok = true;
       int nu = 0;
       // O += P V for the tile issued one step earlier
@@ -438,15 +450,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
         const int pb = it_prev & 1;
         if (!mbar_wait_bounded(&p_full[pb], (it_prev >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t p_hi = p_base + pb * 2 * Tr::kPBytes;
-        const uint32_t p_lo = p_hi + Tr::kPBytes;
+        const uint32_t p_hi = tmem_base + Tr::kPCol + (uint32_t)(pb * 64);
+        const uint32_t p_lo = p_hi + 32;
         const uint32_t v_base = smem_addr(smem + stage_prev * Tr::kStageBytes + Tr::kTileBytes);
 #pragma unroll
-        for (int k = 0; k < kTcTile / 16; ++k) {
+        for (int k = 0; k < kTcTile / 16; ++k) {  // 16 tokens = 8 columns of packed pairs
           const uint64_t b = umma_desc_sw128(v_base + k * 16 * 128, Tr::kSlabBytes, 1024);
-          umma_f16(tmem_base + Tr::kOCol, umma_desc_sw128(p_hi + k * 32, 16, 1024), b, kIdescO,
-                   (first_prev && k == 0) ? 0u : 1u);
-          umma_f16(tmem_base + Tr::kOCol, umma_desc_sw128(p_lo + k * 32, 16, 1024), b, kIdescO, 1u);
+          umma_f16_tmem_a(tmem_base + Tr::kOCol, p_hi + 8 * k, b, kIdescO, (first_prev && k == 0) ? 0u : 1u);
+          umma_f16_tmem_a(tmem_base + Tr::kOCol, p_lo + 8 * k, b, kIdescO, 1u);
         }
         umma_commit(&empty[stage_prev]);
         umma_commit(&o_done[pb]);
@@ -658,23 +669,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
         l = 0.f;
       }
 
-      // P = 2^(x - m_ref) as high + low 16-bit parts, row r of the 128B-swizzled slab
-      unsigned char* phi = smem + Tr::kPOffset + sb * 2 * Tr::kPBytes + r * 128;
-      unsigned char* plo = phi + Tr::kPBytes;
+      // P = 2^(x - m_ref) as high + low 16-bit parts, written to this row's tensor-memory
+      // lane: packed pairs, tokens 2c and 2c + 1 in column c
+      uint32_t hi[kTcTile / 2], lo[kTcTile / 2];
 #pragma unroll
-      for (int ch = 0; ch < kTcTile / 8; ++ch) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int c = 8 * ch + 2 * k;
-          const float p0 = x[c] == -INFINITY ? 0.f : ex2_fast(x[c] - m_ref);
-          const float p1 = x[c + 1] == -INFINITY ? 0.f : ex2_fast(x[c + 1] - m_ref);
-          l += p0 + p1;
-          split_pair<T>(p0, p1, hi[k], lo[k]);
-        }
-        const int sw = (ch ^ (r & 7)) << 4;
-        *reinterpret_cast<uint4*>(phi + sw) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(plo + sw) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      for (int c2 = 0; c2 < kTcTile / 2; ++c2) {
+        const int c = 2 * c2;
+        const float p0 = x[c] == -INFINITY ? 0.f : ex2_fast(x[c] - m_ref);
+        const float p1 = x[c + 1] == -INFINITY ? 0.f : ex2_fast(x[c + 1] - m_ref);
+        l += p0 + p1;
+        split_pair<T>(p0, p1, hi[c2], lo[c2]);
+      }
+      {
+        const uint32_t pcol = trow + Tr::kPCol + (uint32_t)(sb * 64);
+        tmem_st16(pcol, *reinterpret_cast<uint32_t(*)[16]>(hi));
+        tmem_st16(pcol + 16, *reinterpret_cast<uint32_t(*)[16]>(hi + 16));
+        tmem_st16(pcol + 32, *reinterpret_cast<uint32_t(*)[16]>(lo));
+        tmem_st16(pcol + 48, *reinterpret_cast<uint32_t(*)[16]>(lo + 16));
+        tmem_wait_st();
       }
       // V rows past the tile's valid tokens may hold anything (NaN in unwritten
       // slots): zero them so that 0 * V stays 0
@@ -688,7 +700,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
               make_uint4(0, 0, 0, 0);
         }
       }
-      fence_proxy_async_smem();  // P and the zeroed rows are read by the tensor cores
+      if (n_valid < kTcTile) fence_proxy_async_smem();  // the zeroed rows are read by the tensor cores
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[sb]);
