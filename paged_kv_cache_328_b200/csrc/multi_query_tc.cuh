@@ -44,6 +44,7 @@ constexpr int kTcRows = 128;          // M: query rows per tile = tensor-memory 
 constexpr int kTcTile = 64;           // tokens per K/V tile
 constexpr int kTcStages = 6;  // the P V product of tile t is issued after S of tile t + 2
 constexpr int kTcThreads = 6 * 32;    // producer, MMA, four softmax warps
+constexpr int kTcCtasPerSm = 1;       // shared memory (and tensor memory) per CTA
 constexpr int kTcTmemCols = 512;      // S[2] at columns 0 and 64, O at 128, P[2] (high, low) at 256 and 320
 constexpr float kTcRescaleLog2 = 8.0f;
 

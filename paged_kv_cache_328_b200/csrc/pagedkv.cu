@@ -375,7 +375,7 @@ int launch_tc(const pkv::TcParams& prm, long long max_units, cudaStream_t st) {
     }
   }
   if (sms <= 0) return PKV_ECUDA;
-  long long grid = sms;  // one CTA per SM (shared memory and tensor memory)
+  long long grid = (long long)sms * pkv::kTcCtasPerSm;  // resident CTAs (shared memory and tensor memory)
   if (grid > max_units) grid = max_units;
   if (grid < 1) grid = 1;
   cudaLaunchConfig_t cfg = {};
