@@ -549,7 +549,11 @@ def run_gpu(a, rank, world, local_rank):
 def run_reference(a, rank, world):
     if rank != 0:
         return
-    n_seq = {"opt13b": 4, "llama7b": 16, "cow": 4, "longctx": 1, "tiny": 4}[a.workload]
+    if a.workload == "swap":
+        print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the oracle's attention; "
+                          "the swap workload has no attention step"}), flush=True)
+        return
+    n_seq = {"opt13b": 4, "llama7b": 16, "cow": 4, "longctx": 1, "tiny": 4}.get(a.workload, 4)
     sample = make_cpu_sample(a.workload, a.block_size, n_seq=n_seq)
     pool, cores = start_cpu_pool(sample)
     for _ in range(a.warmup):
