@@ -158,3 +158,19 @@ def test_wait_selftest_rejects_limits_on_host(lib):
     assert lib.pkv_selftest_wait_timeout(0, None) == PKV_EINVAL
     assert lib.pkv_selftest_wait_timeout(-5, None) == PKV_EINVAL
     assert lib.pkv_selftest_wait_timeout(2_000_000_001, None) == PKV_EINVAL
+
+
+def test_multi_query_plan_counts_128_row_tiles_above_16_rows(lib):
+    # 32 query rows per K/V head (Lq = 32, G = 1) run on the tcgen05 kernel's 128-row tiles:
+    # 100 sequences x 8 K/V heads x 1 tile = 800 units < 4 x 296, so contexts up to 2048 are split
+    # into 512-token partitions (with 16-row tiles it would be 1600 units and no split)
+    S, Lq, H, Hkv, D, B, MB = 100, 32, 8, 8, 128, 16, 128
+    P, rows = 4, Lq * H
+    split = 16 + S * P * 8 + S * rows * P * 8 + S * rows * P * D * 4
+    assert lib.paged_attn_multi_query_workspace_size(S, Lq, H, Hkv, D, B, MB, 0) == split
+    # 16 rows per K/V head (Lq = 2, G = 8) stay on 16-row tiles: 800 units as well, split
+    P, rows = 4, 2 * 64
+    assert lib.paged_attn_multi_query_workspace_size(S, 2, 64, 8, D, B, MB, 0) == \
+        16 + S * P * 8 + S * rows * P * 8 + S * rows * P * D * 4
+    # enough units for no split: 200 sequences x 8 K/V heads x 1 tile = 1600
+    assert lib.paged_attn_multi_query_workspace_size(200, 32, 8, 8, D, B, MB, 0) == 16 + 200 * 8
