@@ -25,3 +25,32 @@ def test_c_program_against_the_library(tmp_path):
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0, run.stderr + run.stdout
     assert "C ABI checks passed" in run.stdout
+
+
+CUDA = "/usr/local/cuda"
+
+
+def build_device_program(tmp_path):
+    builder.build()
+    lib_dir = os.path.dirname(builder.LIB)
+    exe = tmp_path / "abi_device"
+    cmd = ["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+           "-I", os.path.join(CUDA, "include"), os.path.join(ROOT, "tests", "c", "abi_device.c"),
+           "-L", lib_dir, "-lpagedkv", "-L", os.path.join(CUDA, "lib64"), "-lcudart",
+           f"-Wl,-rpath,{lib_dir}", f"-Wl,-rpath,{os.path.join(CUDA, 'lib64')}", "-o", str(exe)]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    return exe
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None or not os.path.isdir(CUDA), reason="gcc and the CUDA toolkit")
+def test_c_device_program_builds(tmp_path):
+    build_device_program(tmp_path)
+
+
+@pytest.mark.gpu
+def test_c_device_program_runs(tmp_path):
+    exe = build_device_program(tmp_path)
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stderr + run.stdout
+    assert "C device path checks passed" in run.stdout
