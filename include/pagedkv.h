@@ -421,7 +421,10 @@ int pkv_abi_version(void);
  *    must start at zero (the work counter) itself, and the array keeps the last
  *    call's contents.  Calls whose kernels overlap on the GPU (other streams,
  *    other host threads) race on the array: order them on one stream.
- *  - Return codes and device-side checks are those of paged_attn_decode.
+ *  - Return codes and device-side checks are those of paged_attn_decode given a
+ *    workspace of PKV_NOALLOC_SCRATCH_BYTES: the same argument checks run in the
+ *    same order (dtype, sizes, scale, then pointers and alignment; num_seqs = 0
+ *    returns PKV_OK after the size checks), and PKV_EWORKSPACE comes last.
  */
 #define PKV_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 int paged_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,

@@ -77,13 +77,22 @@ class BlockManager:
             self.ref[b] += 1
         self.seqs[child] = {"tokens": p["tokens"], "table": list(p["table"])}
 
-    def _append_needs(self, seq):
-        """Free blocks one append of `seq` takes (new block, or copy of a shared last block)."""
-        s = self.seqs[seq]
-        pos = s["tokens"]
-        if pos // self.B == len(s["table"]):
-            return 1
-        return 1 if self.ref[s["table"][pos // self.B]] > 1 else 0
+    def _batch_needs(self, seqs):
+        """Free blocks a batch of appends takes, counted by playing the batch out on
+        reference counts alone: a sequence whose last block is full takes a new one;
+        a write into a last block that still has another holder copies it and drops
+        one holder, so the last of several writers of one block writes in place."""
+        ref = list(self.ref)
+        need = 0
+        for q in seqs:
+            s = self.seqs[q]
+            j = s["tokens"] // self.B
+            if j == len(s["table"]):
+                need += 1
+            elif ref[s["table"][j]] > 1:
+                ref[s["table"][j]] -= 1
+                need += 1
+        return need
 
     def append_tokens(self, seqs):
         """One new token for each listed sequence: returns (slots, cow_pairs)."""
@@ -92,7 +101,7 @@ class BlockManager:
                 raise BlockManagerError("unknown sequence")
         if len(set(seqs)) != len(seqs):
             raise BlockManagerError("repeated sequence")
-        if sum(self._append_needs(q) for q in seqs) > len(self.free):
+        if self._batch_needs(seqs) > len(self.free):
             raise BlockManagerError("no free block")
         slots, pairs = [], []
         for q in seqs:

@@ -52,11 +52,11 @@ struct pkv_block_manager {
   void release(int32_t b) {
     if (--ref[b] == 0) free_list.push_back(b);
   }
-  // free blocks one append of `s` takes: a new block, or the copy of a shared last block
-  int append_needs(const Seq& s) const {
+  // The partly filled last block an append of `s` writes into, or -1 when the
+  // append starts a new block.
+  int32_t write_block(const Seq& s) const {
     const int64_t j = s.tokens / block_size;
-    if (j == (int64_t)s.table.size()) return 1;
-    return ref[s.table[j]] > 1 ? 1 : 0;
+    return j == (int64_t)s.table.size() ? -1 : s.table[j];
   }
 };
 
@@ -134,12 +134,26 @@ int pkv_bm_append_tokens(pkv_block_manager* bm, const int64_t* seqs, int n, int6
   if (!bm || n < 0 || (n > 0 && (!seqs || !slots || !cow_pairs)) || !num_pairs) return PKV_EINVAL;
   Lock lk(bm->mu);
   *num_pairs = 0;
+  // Free blocks the batch takes: one per sequence whose last block is full, plus
+  // the copies of shared last blocks.  The writers of one shared block b are
+  // served in order: each copies while b still has another holder, so k writers
+  // of a block with r holders make min(k, r - 1) copies (when all r holders write,
+  // the last one writes in place).
   std::unordered_set<int64_t> seen;
+  std::unordered_map<int32_t, int64_t> writers;
   int64_t need = 0;
   for (int i = 0; i < n; ++i) {
     auto it = bm->seqs.find(seqs[i]);
     if (it == bm->seqs.end() || !seen.insert(seqs[i]).second) return PKV_ESEQ;
-    need += bm->append_needs(it->second);
+    const int32_t b = bm->write_block(it->second);
+    if (b < 0)
+      ++need;
+    else if (bm->ref[b] > 1)
+      ++writers[b];
+  }
+  for (const auto& kv : writers) {
+    const int64_t holders = bm->ref[kv.first];
+    need += kv.second < holders - 1 ? kv.second : holders - 1;
   }
   if (need > (int64_t)bm->free_list.size()) return PKV_ENOMEM;
   int pairs = 0;

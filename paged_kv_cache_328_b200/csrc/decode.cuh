@@ -37,9 +37,10 @@
 //       M = max_p m_p,  L = sum_p l_p 2^(m_p - M),  out = sum_p acc_p 2^(m_p - M) / L,
 //     which is exact algebra.
 //
-// "Gather the non-contiguous blocks along the block table and compute
-// softmax(QK^T)V" ("PagedAttention - Efficient Memory Management for LLM Serving
-// with vLLM", section "Method (PagedAttention + vLLM)"): the gather is done by the
+// The method follows each sequence's block table to its scattered physical blocks
+// and attends over them as if they were one contiguous context
+// ("PagedAttention - Efficient Memory Management for LLM Serving with vLLM",
+// section "Method (PagedAttention + vLLM)").  Here the gather is done by the
 // copy engine straight into shared memory, so each K/V byte crosses HBM once.
 // One query per sequence makes this ~1 flop per byte: HBM-bound, no tensor cores.
 #pragma once

@@ -996,16 +996,23 @@ extern "C" int paged_attn_decode_noalloc(const void* q, const void* k_cache, con
                                          int num_heads, int head_dim, int block_size, int max_blocks_per_seq,
                                          int num_blocks, pkv_dtype dtype, float scale, float* out,
                                          int partition_tokens, void* stream) {
-  const size_t need = paged_attn_decode_workspace_size(num_seqs, num_heads, head_dim, block_size,
-                                                       max_blocks_per_seq, partition_tokens);
-  if (need == (size_t)-1) {
-    // the same argument error paged_attn_decode reports
-    DecodePlan plan;
-    return make_plan(num_seqs, num_heads, num_heads, head_dim, block_size, max_blocks_per_seq, partition_tokens,
-                     &plan);
-  }
-  if (need > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_EWORKSPACE;
+  // The argument checks of paged_attn_decode, in its order, so that both entry
+  // points return the same code for the same arguments; the scratch array then
+  // plays the part of a caller workspace of PKV_NOALLOC_SCRATCH_BYTES.
+  if (elem_bytes(dtype) == 0) return PKV_EDTYPE;
+  if (num_heads <= 0) return PKV_EINVAL;
+  DecodePlan plan;
+  const int prc = make_plan(num_seqs, num_heads, num_heads, head_dim, block_size, max_blocks_per_seq,
+                            partition_tokens, &plan);
+  if (prc != PKV_OK) return prc;
+  if (num_blocks <= 0) return PKV_EINVAL;
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return PKV_EINVAL;
   if (num_seqs == 0) return PKV_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PKV_EINVAL;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return PKV_EALIGN;
+  if (plan.bytes > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_EWORKSPACE;
   void* scratch = nullptr;
   const int rc = noalloc_scratch(&scratch);
   if (rc != PKV_OK) return rc;

@@ -174,3 +174,39 @@ def test_multi_query_plan_counts_128_row_tiles_above_16_rows(lib):
         16 + S * P * 8 + S * rows * P * 8 + S * rows * P * D * 4
     # enough units for no split: 200 sequences x 8 K/V heads x 1 tile = 1600
     assert lib.paged_attn_multi_query_workspace_size(200, 32, 8, 8, D, B, MB, 0) == 16 + 200 * 8
+
+
+# Each case has one defect that the host checks catch before any CUDA call, so no
+# pointer is ever used; "big" sizes need more than the 32 MiB scratch array.
+_SMALL = dict(S=4, H=2, D=64, B=16, MB=4, NB=16, dt=1, scale=0.125, pt=0, q=0x10000, out=0x10000)
+_BIG = dict(_SMALL, S=64, H=64, D=128, MB=2048, pt=16)
+_CASES = {
+    "bad dtype, big sizes": (dict(_BIG, dt=7), PKV_EDTYPE),
+    "bad dtype, no sequences": (dict(_SMALL, S=0, dt=7), PKV_EDTYPE),
+    "no sequences": (dict(_SMALL, S=0), PKV_OK),
+    "no sequences, big sizes": (dict(_BIG, S=0), PKV_OK),
+    "no heads": (dict(_SMALL, H=0), PKV_EINVAL),
+    "head_dim 80": (dict(_SMALL, D=80), PKV_EUNSUPPORTED),
+    "block size 24": (dict(_SMALL, B=24), PKV_EUNSUPPORTED),
+    "partition not a multiple of B": (dict(_SMALL, pt=17), PKV_EINVAL),
+    "no blocks, big sizes": (dict(_BIG, NB=0), PKV_EINVAL),
+    "nan scale, big sizes": (dict(_BIG, scale=float("nan")), PKV_EINVAL),
+    "null q, big sizes": (dict(_BIG, q=0), PKV_EINVAL),
+    "misaligned out, big sizes": (dict(_BIG, out=0x10004), PKV_EALIGN),
+    "big sizes": (_BIG, PKV_EWORKSPACE),
+}
+
+
+@pytest.mark.parametrize("name", sorted(_CASES))
+def test_noalloc_returns_what_decode_returns(lib, name):
+    """The allocation-free decode runs the argument checks of paged_attn_decode in
+    the same order, with its scratch array standing in for a workspace of
+    PKV_NOALLOC_SCRATCH_BYTES: both return the same code for the same arguments."""
+    a, want = _CASES[name]
+    fake = 0x10000
+    common = (a["q"], fake, fake, fake, fake, a["S"], a["H"], a["D"], a["B"], a["MB"], a["NB"], a["dt"],
+              ctypes.c_float(a["scale"]), a["out"], a["pt"])
+    got_noalloc = lib.paged_attn_decode_noalloc(*common, None)
+    got_decode = lib.paged_attn_decode(*common, 0x20000, _lib.NOALLOC_SCRATCH_BYTES, None)
+    assert got_decode == want, (name, got_decode)
+    assert got_noalloc == want, (name, got_noalloc)

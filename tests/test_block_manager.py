@@ -120,3 +120,29 @@ def test_error_codes_and_no_change():
     assert e.value.code == PKV_ESEQ
     tables, lens = bm.fill_tables([1, 0], 4)
     assert tables.tolist() == [[2, -1, -1, -1], [0, 1, -1, -1]] and lens.tolist() == [3, 8]
+
+
+@pytest.mark.parametrize("holders,free,writers", [(2, 1, 2), (3, 2, 3), (3, 1, 2), (3, 2, 2), (4, 2, 4),
+                                                   (4, 3, 4), (2, 0, 2), (2, 0, 1)])
+def test_shared_last_block_batches_agree(holders, free, writers):
+    """Forks sharing a partly filled last block append together: k writers of a
+    block with r holders take min(k, r - 1) free blocks; native and model agree on
+    success, slots, pairs and state, and on refusing batches that do not fit."""
+    nb = 2 + free
+    impls = [pkv.BlockManager(nb, 4), oracle.BlockManager(nb, 4)]
+    for bm in impls:
+        bm.add_sequence(0, 6)
+        for c in range(1, holders):
+            bm.fork(0, c)
+    batch = list(range(holders))[::-1][:writers]
+    got = []
+    for bm in impls:
+        try:
+            slots, pairs = bm.append_tokens(batch)
+            got.append((list(slots), [tuple(p) for p in pairs]))
+        except (oracle.BlockManagerError, pkv.PagedKVError):
+            got.append("refused")
+    assert got[0] == got[1]
+    fits = min(writers, holders - 1) <= free
+    assert (got[0] != "refused") == fits
+    same_state(impls[0], impls[1], nb)

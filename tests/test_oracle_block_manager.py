@@ -79,6 +79,42 @@ def test_out_of_blocks_changes_nothing():
     check_invariants(bm, 3)
 
 
+def test_siblings_sharing_a_last_block_need_one_copy():
+    """Two forks that share a partly filled last block append in one batch: the
+    first copies it (copy-on-write), after which the block has one holder left and
+    the second writes in place, so one free block serves the batch.  Worked out by
+    hand: B = 4, FIFO order 0, 1, 2, ..."""
+    bm = BlockManager(3, 4)
+    bm.add_sequence(0, 6)                      # blocks [0, 1], 2 tokens in block 1
+    bm.fork(0, 1)                              # blocks 0 and 1 held twice
+    assert bm.num_free() == 1
+    slots, pairs = bm.append_tokens([0, 1])
+    assert pairs == [(1, 2)]                   # seq 0 copies block 1 into block 2
+    assert slots == [2 * 4 + 2, 1 * 4 + 2]     # seq 1 writes block 1 in place
+    assert bm.block_table(0) == ([0, 2], 7) and bm.block_table(1) == ([0, 1], 7)
+    assert bm.ref == [2, 1, 1] and bm.num_free() == 0
+    check_invariants(bm, 3)
+    # three holders, two free blocks: two copies, the last writer in place
+    bm = BlockManager(4, 4)
+    bm.add_sequence(0, 6)
+    bm.fork(0, 1)
+    bm.fork(0, 2)
+    slots, pairs = bm.append_tokens([2, 0, 1])
+    assert pairs == [(1, 2), (1, 3)] and slots == [10, 14, 6]
+    assert bm.num_free() == 0
+    check_invariants(bm, 4)
+    # three holders, one free block: two of them writing need two copies (the
+    # block keeps a third holder), so the batch is refused and nothing changes
+    bm = BlockManager(3, 4)
+    bm.add_sequence(0, 6)
+    bm.fork(0, 1)
+    bm.fork(0, 2)
+    with pytest.raises(BlockManagerError):
+        bm.append_tokens([0, 1])
+    assert bm.ref == [3, 3, 0] and bm.num_free() == 1
+    check_invariants(bm, 3)
+
+
 def test_random_operations_keep_invariants():
     rng = random.Random(5)
     nb = 40

@@ -9,7 +9,8 @@ inside the library instead of a caller workspace.
 These tests call that entry point through the C ABI (ctypes, no Python wrapper),
 twice in a row on different inputs, so that the second call starts from the
 scratch contents the first one left behind, and compare each output with the
-ordinary entry point's output on the same inputs.  The file is named so that
+CPU oracle (float64, from host copies of the inputs) and with the ordinary
+entry point's output on the same inputs.  The file is named so that
 pytest collects it after every other test file; it also passes on its own in a
 fresh process (the first call on a device does the scratch set-up).
 """
@@ -20,6 +21,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import paged_kv_cache_328_b200 as pkv
 from paged_kv_cache_328_b200 import _lib
 from paged_kv_cache_328_b200 import workloads as wl
@@ -53,6 +55,8 @@ def test_noalloc_matches_the_workspace_entry_point_on_two_calls_in_a_row():
     for w, pt in cases:
         bt = torch.from_numpy(w.block_tables).to(dev)
         ctx = torch.from_numpy(w.context_lens).to(dev)
+        want = oracle.paged_decode(w.host(w.q), w.host(w.k_pool), w.host(w.v_pool), w.block_tables,
+                                   w.context_lens, w.scale, w.B, w.dtype)
         ref = pkv.paged_attn_decode(w.q, w.k_pool, w.v_pool, bt, ctx, w.scale, partition_tokens=pt)
         out = torch.full((w.S, w.H, w.D), float("nan"), dtype=torch.float32, device=dev)
         assert _lib.workspace_size(w.S, w.H, w.D, w.B, w.max_blocks, pt) <= _lib.NOALLOC_SCRATCH_BYTES
@@ -61,7 +65,9 @@ def test_noalloc_matches_the_workspace_entry_point_on_two_calls_in_a_row():
         code, reason = pkv.get_device_error(dev)
         assert code == 0, (code, reason)
         assert bool(torch.isfinite(out).all())
+        assert max_err(out.cpu(), want) <= TOL[w.dtype]
         assert max_err(out.cpu(), ref.cpu().numpy()) <= TOL[w.dtype]
+        assert np.all(out.cpu().numpy()[w.context_lens == 0] == 0.0)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
