@@ -59,7 +59,10 @@ typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
 /* Return codes. */
 enum {
   PKV_OK = 0,
-  PKV_EINVAL = -1,        /* a null pointer, a negative or too-large size, bad partition size */
+  PKV_EINVAL = -1,        /* a null pointer, a negative or too-large size, bad partition size;
+                             attention calls also reject num_seqs > 65535, (query tokens x) query
+                             heads > 65535 and more than 32767 partitions per sequence (a work
+                             unit packs the sequence and partition indices into 16 bits each) */
   PKV_EDTYPE = -2,        /* dtype is not a pkv_dtype */
   PKV_EALIGN = -3,        /* a pointer is not aligned as required */
   PKV_EUNSUPPORTED = -4,  /* head_dim or block_size not in the supported set */
@@ -68,7 +71,8 @@ enum {
   PKV_EDEVICE = -7,       /* a kernel flagged bad device data (see pkv_get_device_error) */
   PKV_ETIMEOUT = -8,      /* a kernel's bounded wait ran out (see pkv_get_device_error) */
   PKV_ENOMEM = -9,        /* block manager: not enough free blocks (nothing was changed) */
-  PKV_ESEQ = -10          /* block manager: unknown sequence, sequence exists, or repeated in a batch */
+  PKV_ESEQ = -10,         /* block manager: unknown sequence, sequence exists, or repeated in a batch */
+  PKV_EOVERLAP = -11      /* debug checks: copy pairs overlap, or two appended tokens share a slot */
 };
 
 /* Reasons stored in the device error word (the `reason` of pkv_get_device_error). */
@@ -252,7 +256,10 @@ size_t paged_attn_multi_query_workspace_size(int num_seqs, int q_len, int num_he
  * ("LLM Inference 8 - PagedAttention", section "KV Cache의 메모리 문제": the new
  * token's Key and Value are added to the cache.)  slot = -1 skips the token; a
  * slot >= num_blocks * B is skipped and flagged (PKV_DEV_SLOT).  Two tokens
- * with the same slot race (unspecified which one lands).  Bit-exact copy.
+ * with the same slot race (unspecified which one lands) unless debug checks are
+ * on (pkv_set_debug_checks): then the call copies slot_mapping to the host,
+ * synchronising the stream, and returns PKV_EOVERLAP without launching when
+ * pkv_check_slots rejects it.  Bit-exact copy.
  *
  *   k, v          [num_tokens][num_heads][head_dim], storage dtype.
  *   slot_mapping  int64 [num_tokens].
@@ -270,15 +277,41 @@ int kv_cache_append(const void* k, const void* v, void* k_cache, void* v_cache,
  * (all heads, all block_size slots).  ("PagedAttention - Efficient Memory
  * Management for LLM Serving with vLLM", section "Method (PagedAttention +
  * vLLM)", copy-on-write: only the written block is copied.)  Pairs must not
- * overlap: no dst may repeat or appear as any src, and src != dst; overlapping
- * pairs race.  A pair with an id outside [0, num_blocks) is skipped and flagged
- * (PKV_DEV_COPY_PAIR).  Bit-exact copy.
+ * overlap: no dst may repeat or appear as any src, and src != dst (a copy always
+ * fills a fresh block, as in the digest's flowchart: P3 -> P9); one src may feed
+ * several dsts.  Overlapping pairs race unless debug checks are on
+ * (pkv_set_debug_checks): then the call copies the pairs to the host,
+ * synchronising the stream, and returns PKV_EOVERLAP without launching when
+ * pkv_check_copy_pairs rejects them.  A pair with an id outside [0, num_blocks)
+ * is skipped and flagged (PKV_DEV_COPY_PAIR).  Bit-exact copy.
  *
  *   src_dst_pairs int64 [num_pairs][2], device memory.
  */
 int kv_block_copy(void* k_cache, void* v_cache, const int64_t* src_dst_pairs,
                   int num_pairs, int num_heads, int head_dim, int block_size,
                   int num_blocks, pkv_dtype dtype, void* stream);
+
+/*
+ * Overlap checks of the cache-maintenance inputs, on host arrays (no CUDA call).
+ *
+ * pkv_check_copy_pairs: PKV_EOVERLAP if some pair has src == dst, some dst
+ *   appears twice, or some dst is also a src; else PKV_OK.  Pairs with a
+ *   negative id copy nothing and are ignored.  host_pairs is int64
+ *   [num_pairs][2] (src, dst) in host memory.
+ * pkv_check_slots: PKV_EOVERLAP if two tokens have the same slot >= 0; else
+ *   PKV_OK (negative slots skip their token and never collide).
+ * Both return PKV_EINVAL for num < 0 or a null array with num > 0.
+ *
+ * pkv_set_debug_checks(enable): with enable = 1 (0), kv_block_copy and
+ *   kv_cache_append run these checks on every call (do not); enable < 0 only
+ *   queries.  Returns the setting before the call.  The initial setting is on
+ *   when the environment variable PKV_CHECK is "1" at the first query, else off.
+ *   A checked call synchronises its stream (the indices are device memory), so
+ *   the checks are for debugging, not for a serving loop's hot path.
+ */
+int pkv_check_copy_pairs(const int64_t* host_pairs, int num_pairs);
+int pkv_check_slots(const int64_t* host_slots, int num_tokens);
+int pkv_set_debug_checks(int enable);
 
 /*
  * paged_kv_gather - copy one sequence's cached rows into contiguous memory.

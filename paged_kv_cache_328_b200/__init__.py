@@ -22,6 +22,8 @@ from ._lib import (  # noqa: F401
     PagedKVError,
     abi_version,
     alloc_workspace,
+    check_copy_pairs,
+    check_slots,
     get_device_error,
     gqa_partition_tokens,
     gqa_workspace_size,
@@ -35,6 +37,7 @@ from ._lib import (  # noqa: F401
     paged_kv_gather,
     partition_tokens,
     selftest_wait_timeout,
+    set_debug_checks,
     strerror,
     tune_partition_tokens,
     workspace_size,

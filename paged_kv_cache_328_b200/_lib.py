@@ -20,7 +20,7 @@ DTYPE_CODE = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PK
 ERRORS = {
     0: "PKV_OK", -1: "PKV_EINVAL", -2: "PKV_EDTYPE", -3: "PKV_EALIGN", -4: "PKV_EUNSUPPORTED",
     -5: "PKV_ECUDA", -6: "PKV_EWORKSPACE", -7: "PKV_EDEVICE", -8: "PKV_ETIMEOUT", -9: "PKV_ENOMEM",
-    -10: "PKV_ESEQ",
+    -10: "PKV_ESEQ", -11: "PKV_EOVERLAP",
 }
 DEVICE_REASONS = {0: "ok", 1: "block id", 2: "context length", 3: "slot", 4: "copy pair", 5: "wait timeout"}
 
@@ -67,6 +67,9 @@ SIGNATURES = {
     "pkv_bm_ref_count": (_c_int, [_c_void_p, _c_int]),
     "pkv_bm_swap_out": (_c_int, [_c_void_p, ctypes.c_int64, _c_void_p, _c_int, ctypes.POINTER(_c_int)]),
     "pkv_bm_swap_in": (_c_int, [_c_void_p, ctypes.c_int64, _c_void_p, _c_int, ctypes.POINTER(_c_int)]),
+    "pkv_check_copy_pairs": (_c_int, [_c_void_p, _c_int]),
+    "pkv_check_slots": (_c_int, [_c_void_p, _c_int]),
+    "pkv_set_debug_checks": (_c_int, [_c_int]),
     "paged_attn_decode_noalloc": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                            _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                            _c_float, _c_void_p, _c_int, _c_void_p]),
@@ -250,6 +253,30 @@ def kv_block_copy(k_cache, v_cache, src_dst_pairs, stream=None):
             H, D, B, NB, DTYPE_CODE[k_cache.dtype])
     rc = _call(lib.kv_block_copy, args, k_cache.device, stream)
     _check(rc, "kv_block_copy")
+
+
+def _host_int64(a, name):
+    import numpy as np
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.int64))
+    return a, a.ctypes.data if a.size else None
+
+
+def check_copy_pairs(pairs):
+    """PKV_OK (0) or PKV_EOVERLAP for host (src, dst) pairs [n, 2] (no CUDA call)."""
+    a, ptr = _host_int64(pairs, "pairs")
+    return load().pkv_check_copy_pairs(ptr, a.size // 2)
+
+
+def check_slots(slots):
+    """PKV_OK (0) or PKV_EOVERLAP for a host slot mapping [T] (no CUDA call)."""
+    a, ptr = _host_int64(slots, "slots")
+    return load().pkv_check_slots(ptr, a.size)
+
+
+def set_debug_checks(enable):
+    """Turn the overlap checks of kv_block_copy / kv_cache_append on or off (None:
+    query); returns the previous setting."""
+    return bool(load().pkv_set_debug_checks(-1 if enable is None else (1 if enable else 0)))
 
 
 def paged_kv_gather(cache, block_table_row, context_len, out=None, stream=None):

@@ -5,10 +5,14 @@
 // kernels live in decode.cuh (paged decode attention: plan, persistent decode
 // with the log-sum-exp merge of split contexts) and cache_ops.cuh (append, block
 // copy, gather).
+#include <atomic>
 #include <climits>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <unordered_set>
+#include <vector>
 
 #include <cudaTypedefs.h>
 
@@ -17,6 +21,7 @@
 #include "decode.cuh"
 #include "decode_gqa.cuh"
 #include "multi_query_tc.cuh"
+#include "gqa_tc.cuh"
 #include "cache_ops.cuh"
 
 namespace {
@@ -283,16 +288,33 @@ bool use_gqa_kernel(int Hq, int Hkv, int B, int NB, pkv_dtype dt) {
   return G >= 2 && G <= pkv::kGqaRows && dt != PKV_F32 && (long long)NB * Hkv * B < (1LL << 31);
 }
 
-// More than 16 query rows per K/V head (Lq * G) run on the tcgen05 kernel with
-// 128-row tiles of floor(128 / G) whole query tokens; up to 16 rows on the
-// mma.sync kernel's 16-row tiles.  The choice depends only on the shapes, so the
-// workspace query and the launch agree.
+// Which tensor-core kernel serves Lq * G query rows per K/V head (16-bit K/V):
+//  * kKt: the token-major tcgen05 kernel (gqa_tc.cuh), head_dim 128 and
+//    kKtMinRows < Lq * G <= kKtMaxRows: all rows of a (sequence, K/V head) in one
+//    row tile, the tile's tokens as M;
+//  * kTc128: the row-major tcgen05 kernel (multi_query_tc.cuh) above that (or
+//    head_dim 64 above 16 rows): 128-row tiles of floor(128 / G) whole query tokens;
+//  * kMmaSync: the warp-level kernel (decode_gqa.cuh), 16-row tiles.
+// The choice depends only on the shapes, so the workspace query and the launch agree.
+enum class TcPath { kMmaSync, kKt, kTc128 };
+constexpr long long kKtMinRows = 16;
+constexpr long long kKtMaxRows = 64;
+
+TcPath tc_path(long long q_len, int group, int head_dim) {
+  const long long rows = q_len * group;
+  if (head_dim == 128 && rows > kKtMinRows && rows <= kKtMaxRows) return TcPath::kKt;
+  if (rows > pkv::kGqaRows && group <= pkv::kTcRows && (head_dim == 64 || head_dim == 128)) return TcPath::kTc128;
+  return TcPath::kMmaSync;
+}
+
 bool mq_uses_tcgen05(long long q_len, int group, int head_dim) {
-  return q_len * group > pkv::kGqaRows && group <= pkv::kTcRows && (head_dim == 64 || head_dim == 128);
+  return tc_path(q_len, group, head_dim) != TcPath::kMmaSync;
 }
 
 long long mq_row_tiles(long long q_len, int group, int head_dim) {
-  if (mq_uses_tcgen05(q_len, group, head_dim)) {
+  const TcPath path = tc_path(q_len, group, head_dim);
+  if (path == TcPath::kKt) return 1;
+  if (path == TcPath::kTc128) {
     const long long tq = pkv::kTcRows / group;
     return (q_len + tq - 1) / tq;
   }
@@ -430,6 +452,83 @@ int launch_tcgen05(const void* q, const void* k_cache, const void* v_cache, cons
   return head_dim == 64 ? launch_tc<__half, 64>(t, max_units, st) : launch_tc<__half, 128>(t, max_units, st);
 }
 
+template <typename T, int NR>
+int launch_kt(const pkv::TcParams& prm, long long max_units, cudaStream_t st) {
+  using Tr = pkv::KtTraits<NR>;
+  static bool attr_set[kMaxDevices];
+  int dev;
+  if (current_device(&dev) != PKV_OK) return PKV_ECUDA;
+  const int sms = sm_count(dev);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(pkv::paged_gqa_tc_kernel<T, NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Tr::kSmemAlloc) != cudaSuccess)
+        return PKV_ECUDA;
+      attr_set[dev] = true;
+    }
+  }
+  if (sms <= 0) return PKV_ECUDA;
+  long long grid = sms;  // one CTA per SM (shared memory)
+  if (grid > max_units) grid = max_units;
+  if (grid < 1) grid = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(pkv::kKtThreads);
+  cfg.dynamicSmemBytes = Tr::kSmemAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, pkv::paged_gqa_tc_kernel<T, NR>, prm) != cudaSuccess) return PKV_ECUDA;
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+// The token-major tcgen05 kernel: all Lq * G <= 64 rows of a (sequence, K/V head)
+// in one row tile of NR = 16, 32 or 64 rows; 128-token K/V tiles.
+int launch_kt_path(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables, int num_seqs,
+                   int q_len, int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                   int num_blocks, pkv_dtype dtype, float scale_log2, float* out, const DecodePlan& plan,
+                   const pkv::DecodeParams& prm, cudaStream_t st) {
+  static_assert(alignof(pkv::TcParams) >= 64, "tensor maps need 64-byte alignment");
+  pkv::TcParams t;
+  const int G = num_heads / num_kv_heads;
+  const int rows = q_len * G;
+  const long long pool_rows = (long long)num_blocks * num_kv_heads * block_size;
+  const int box_rows = block_size < pkv::kKtTile ? block_size : pkv::kKtTile;
+  if (encode_pool_map(&t.tmap_k, k_cache, pool_rows, head_dim, box_rows, dtype) != PKV_OK ||
+      encode_pool_map(&t.tmap_v, v_cache, pool_rows, head_dim, box_rows, dtype) != PKV_OK ||
+      encode_query_map(&t.tmap_q, q, num_seqs, q_len, num_heads, head_dim, G, q_len, dtype) != PKV_OK)
+    return PKV_ECUDA;
+  t.block_tables = block_tables;
+  t.num_heads = num_heads;
+  t.num_kv_heads = num_kv_heads;
+  t.group = G;
+  t.q_len = q_len;
+  t.tq_per_tile = q_len;
+  t.row_tiles = 1;
+  t.block_size = block_size;
+  t.max_blocks = max_blocks_per_seq;
+  t.num_blocks = num_blocks;
+  t.scale_log2 = scale_log2;
+  t.part_tokens = plan.part_tokens;
+  t.max_parts = plan.max_parts;
+  t.out = out;
+  t.ws_acc = prm.ws_acc;
+  t.ws_ml = prm.ws_ml;
+  t.units = prm.units;
+  t.counters = prm.counters;
+  const long long max_units = (long long)num_seqs * num_kv_heads * plan.max_parts;
+  const bool bf = dtype == PKV_BF16;
+  if (rows <= 16)
+    return bf ? launch_kt<__nv_bfloat16, 16>(t, max_units, st) : launch_kt<__half, 16>(t, max_units, st);
+  if (rows <= 32)
+    return bf ? launch_kt<__nv_bfloat16, 32>(t, max_units, st) : launch_kt<__half, 32>(t, max_units, st);
+  return bf ? launch_kt<__nv_bfloat16, 64>(t, max_units, st) : launch_kt<__half, 64>(t, max_units, st);
+}
+
 // The merge is a programmatic dependent of the decode kernel: its CTAs may be
 // scheduled as decode CTAs run out of units and wait for the decode to finish.
 template <int D>
@@ -449,6 +548,27 @@ int launch_merge(const int32_t* context_lens, int S, int H, int max_ctx, const D
                          plan.max_parts, ws_acc, ws_ml, out) != cudaSuccess)
     return PKV_ECUDA;
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+// Debug checks of the cache-maintenance inputs: -1 until first queried, then 0 / 1.
+std::atomic<int> g_debug_checks{-1};
+
+bool debug_checks() {
+  int v = g_debug_checks.load();
+  if (v < 0) {
+    const char* e = std::getenv("PKV_CHECK");
+    int want = (e && e[0] == '1' && e[1] == 0) ? 1 : 0;
+    g_debug_checks.compare_exchange_strong(v, want);
+    v = g_debug_checks.load();
+  }
+  return v == 1;
+}
+
+// Copies device (or any CUDA-visible) memory to a host array, in stream order.
+int copy_to_host(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+  if (bytes == 0) return PKV_OK;
+  if (cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault, st) != cudaSuccess) return PKV_ECUDA;
+  return cudaStreamSynchronize(st) == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
 
 int grid_for(long long work, int per_block, int dev) {
@@ -543,7 +663,12 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const i
       context_lens, num_seqs, max_ctx, plan.part_tokens, plan.sort ? 1 : 0,
       reinterpret_cast<uint2*>(ws + plan.off_units), prm.counters);
   if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
-  if (result == PKV_OK && use_gqa_kernel(num_heads, num_kv_heads, block_size, num_blocks, dtype)) {
+  const int group = num_heads / num_kv_heads;
+  const bool tc_ok = dtype != PKV_F32 && group >= 2 && (long long)num_blocks * num_kv_heads * block_size < (1LL << 31);
+  if (result == PKV_OK && tc_ok && tc_path(1, group, head_dim) == TcPath::kKt) {
+    result = launch_kt_path(q, k_cache, v_cache, block_tables, num_seqs, 1, num_heads, num_kv_heads, head_dim,
+                            block_size, max_blocks_per_seq, num_blocks, dtype, prm.scale_log2, out, plan, prm, st);
+  } else if (result == PKV_OK && use_gqa_kernel(num_heads, num_kv_heads, block_size, num_blocks, dtype)) {
     result = launch_tensor_core(q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1, num_heads,
                                 num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, dtype, prm.scale_log2,
                                 out, plan, prm, st);
@@ -616,7 +741,12 @@ int multi_query_impl(const void* q, const void* k_cache, const void* v_cache, co
       context_lens, num_seqs, max_ctx, plan.part_tokens, plan.sort ? 1 : 0,
       reinterpret_cast<uint2*>(ws + plan.off_units), prm.counters);
   if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
-  if (result == PKV_OK && mq_uses_tcgen05(q_len, num_heads / num_kv_heads, head_dim))
+  const TcPath path = tc_path(q_len, num_heads / num_kv_heads, head_dim);
+  if (result == PKV_OK && path == TcPath::kKt)
+    result = launch_kt_path(q, k_cache, v_cache, block_tables, num_seqs, q_len, num_heads, num_kv_heads, head_dim,
+                            block_size, max_blocks_per_seq, num_blocks, dtype, scale * pkv::kLog2e, out, plan, prm,
+                            st);
+  else if (result == PKV_OK && path == TcPath::kTc128)
     result = launch_tcgen05(q, k_cache, v_cache, block_tables, num_seqs, q_len, num_heads, num_kv_heads, head_dim,
                             block_size, max_blocks_per_seq, num_blocks, dtype, scale * pkv::kLog2e, out, plan, prm,
                             st);
@@ -775,6 +905,34 @@ int paged_attn_decode_gqa(const void* q, const void* k_cache, const void* v_cach
                      workspace_bytes, stream);
 }
 
+int pkv_check_copy_pairs(const int64_t* host_pairs, int num_pairs) {
+  if (num_pairs < 0 || (num_pairs > 0 && !host_pairs)) return PKV_EINVAL;
+  std::unordered_set<int64_t> srcs, dsts;
+  for (int i = 0; i < num_pairs; ++i) {
+    if (host_pairs[2 * i] < 0 || host_pairs[2 * i + 1] < 0) continue;  // skipped by the copy kernel
+    srcs.insert(host_pairs[2 * i]);
+    if (host_pairs[2 * i] == host_pairs[2 * i + 1] || !dsts.insert(host_pairs[2 * i + 1]).second)
+      return PKV_EOVERLAP;
+  }
+  for (int64_t d : dsts)
+    if (srcs.count(d)) return PKV_EOVERLAP;
+  return PKV_OK;
+}
+
+int pkv_check_slots(const int64_t* host_slots, int num_tokens) {
+  if (num_tokens < 0 || (num_tokens > 0 && !host_slots)) return PKV_EINVAL;
+  std::unordered_set<int64_t> seen;
+  for (int i = 0; i < num_tokens; ++i)
+    if (host_slots[i] >= 0 && !seen.insert(host_slots[i]).second) return PKV_EOVERLAP;
+  return PKV_OK;
+}
+
+int pkv_set_debug_checks(int enable) {
+  const int before = debug_checks() ? 1 : 0;
+  if (enable >= 0) g_debug_checks.store(enable ? 1 : 0);
+  return before;
+}
+
 int kv_cache_append(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
                     int num_tokens, int num_heads, int head_dim, int block_size, int num_blocks, pkv_dtype dtype,
                     void* stream) {
@@ -793,6 +951,13 @@ int kv_cache_append(const void* k, const void* v, void* k_cache, void* v_cache, 
   const int row_vecs = head_dim * e / 16;
   if ((long long)num_heads * row_vecs > INT_MAX) return PKV_EINVAL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (debug_checks()) {
+    std::vector<int64_t> h((size_t)num_tokens);
+    const int rc = copy_to_host(h.data(), slot_mapping, h.size() * sizeof(int64_t), st);
+    if (rc != PKV_OK) return rc;
+    const int ck = pkv_check_slots(h.data(), num_tokens);
+    if (ck != PKV_OK) return ck;
+  }
   pkv::kv_append_kernel<<<dim3((unsigned)num_tokens, 2), pkv::kAppendThreads, 0, st>>>(
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
       static_cast<uint4*>(v_cache), slot_mapping, num_heads, row_vecs, block_size,
@@ -814,6 +979,13 @@ int kv_block_copy(void* k_cache, void* v_cache, const int64_t* src_dst_pairs, in
   const long long chunks = (block_vecs + per_cta - 1) / per_cta;
   if (chunks > INT_MAX) return PKV_EINVAL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (debug_checks()) {
+    std::vector<int64_t> h(2 * (size_t)num_pairs);
+    const int rc = copy_to_host(h.data(), src_dst_pairs, h.size() * sizeof(int64_t), st);
+    if (rc != PKV_OK) return rc;
+    const int ck = pkv_check_copy_pairs(h.data(), num_pairs);
+    if (ck != PKV_OK) return ck;
+  }
   for (int first = 0; first < num_pairs; first += 65535) {
     const int n = num_pairs - first < 65535 ? num_pairs - first : 65535;
     const dim3 grid((unsigned)chunks, (unsigned)n, 2);
@@ -952,6 +1124,7 @@ const char* pkv_strerror(int code) {
     case PKV_ETIMEOUT: return "a kernel's bounded shared-memory wait ran out";
     case PKV_ENOMEM: return "block manager: not enough free blocks (nothing was changed)";
     case PKV_ESEQ: return "block manager: unknown sequence, sequence already exists, or repeated in a batch";
+    case PKV_EOVERLAP: return "debug checks: copy pairs overlap, or two appended tokens share a slot";
   }
   return "unknown error code";
 }

@@ -210,3 +210,55 @@ def test_noalloc_returns_what_decode_returns(lib, name):
     got_decode = lib.paged_attn_decode(*common, 0x20000, _lib.NOALLOC_SCRATCH_BYTES, None)
     assert got_decode == want, (name, got_decode)
     assert got_noalloc == want, (name, got_noalloc)
+
+
+PKV_EOVERLAP = -11
+
+
+@pytest.mark.parametrize("pairs,want", [
+    ([], PKV_OK),
+    ([[3, 9]], PKV_OK),
+    ([[3, 9], [3, 10], [3, 11]], PKV_OK),            # one shared block forked three times
+    ([[3, 9], [4, 10]], PKV_OK),
+    ([[3, 3]], PKV_EOVERLAP),                        # src == dst
+    ([[3, 9], [4, 9]], PKV_EOVERLAP),                # a dst repeats
+    ([[3, 9], [9, 10]], PKV_EOVERLAP),               # a dst is also a src (chained copy)
+    ([[9, 10], [3, 9]], PKV_EOVERLAP),               # ... in either order
+    ([[-1, 5], [7, -1]], PKV_OK),                    # out-of-range ids are the device's to flag
+])
+def test_check_copy_pairs(lib, pairs, want):
+    import paged_kv_cache_328_b200 as pkv
+    assert pkv.check_copy_pairs(pairs) == want
+
+
+@pytest.mark.parametrize("slots,want", [
+    ([], PKV_OK), ([5, 6, 7], PKV_OK), ([-1, -1, 4], PKV_OK), ([5, 6, 5], PKV_EOVERLAP), ([0, 0], PKV_EOVERLAP),
+])
+def test_check_slots(lib, slots, want):
+    import paged_kv_cache_328_b200 as pkv
+    assert pkv.check_slots(slots) == want
+
+
+def test_check_argument_errors_and_toggle(lib):
+    assert lib.pkv_check_copy_pairs(None, 1) == PKV_EINVAL
+    assert lib.pkv_check_slots(None, -1) == PKV_EINVAL
+    import paged_kv_cache_328_b200 as pkv
+    before = pkv.set_debug_checks(None)
+    assert pkv.set_debug_checks(True) == before
+    assert pkv.set_debug_checks(None) is True
+    assert pkv.set_debug_checks(False) is True
+    assert pkv.set_debug_checks(None) is False
+    pkv.set_debug_checks(before)
+    assert _lib.strerror(PKV_EOVERLAP) != "unknown error code"
+
+
+def test_debug_checks_follow_the_environment():
+    """PKV_CHECK=1 turns the checks on at the first query (a fresh process)."""
+    import subprocess
+    import sys
+    code = ("import paged_kv_cache_328_b200 as p; import sys; "
+            "sys.exit(0 if p.set_debug_checks(None) else 3)")
+    env = dict(os.environ, PKV_CHECK="1")
+    assert subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env).returncode == 0
+    env["PKV_CHECK"] = "0"
+    assert subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env).returncode == 3

@@ -87,6 +87,9 @@ def test_native_matches_model(seed):
                 elif call[0] == "append":
                     slots, pairs = impl.append_tokens(call[1])
                     results.append((list(slots), [tuple(p) for p in pairs]))
+                    # a step's outputs never overlap: they pass the debug checks
+                    assert pkv.check_slots(list(slots)) == 0
+                    assert pkv.check_copy_pairs([list(p) for p in pairs]) == 0
                 elif call[0] == "free":
                     impl.free_sequence(call[1])
                     results.append(None)

@@ -184,3 +184,41 @@ def test_bad_block_id_and_context_are_flagged(dev):
                                w.context_lens, w.scale, w.B, w.dtype)
     assert float(np.max(np.abs(out.cpu().numpy() - want))) <= 2e-3
     clean(dev)
+
+
+def test_debug_checks_reject_overlaps_before_launch(dev):
+    """With the debug checks on, overlapping copy pairs and duplicate append slots
+    are rejected on the host (PKV_EOVERLAP) and the pools are left untouched;
+    valid inputs still copy bit-exactly."""
+    nb, H, B, D = 16, 2, 16, 128
+    kc, vc = nan_pool(nb, H, B, D, "bf16", dev, 21), nan_pool(nb, H, B, D, "bf16", dev, 22)
+    k0, v0 = host(kc), host(vc)
+    before = pkv.set_debug_checks(True)
+    try:
+        for bad in ([[2, 2]], [[1, 7], [3, 7]], [[1, 7], [7, 9]]):
+            with pytest.raises(pkv.PagedKVError) as e:
+                pkv.kv_block_copy(kc, vc, torch.tensor(bad, dtype=torch.int64, device=dev))
+            assert e.value.code == -11, bad
+        g = torch.Generator(device=dev)
+        g.manual_seed(23)
+        k = torch.randn((3, H, D), generator=g, device=dev).to(torch.bfloat16)
+        v = torch.randn((3, H, D), generator=g, device=dev).to(torch.bfloat16)
+        with pytest.raises(pkv.PagedKVError) as e:
+            pkv.kv_cache_append(k, v, kc, vc, torch.tensor([5, 40, 5], dtype=torch.int64, device=dev))
+        assert e.value.code == -11
+        torch.cuda.synchronize()
+        assert np.array_equal(host(kc), k0) and np.array_equal(host(vc), v0)
+        # one source forked into three fresh blocks passes, and copies bit-exactly
+        pairs = np.array([[4, 10], [4, 11], [5, 12]], dtype=np.int64)
+        pkv.kv_block_copy(kc, vc, torch.from_numpy(pairs).to(dev))
+        ke, ve, nbad = oracle.kv_block_copy(k0, v0, pairs)
+        assert nbad == 0
+        assert np.array_equal(host(kc), ke) and np.array_equal(host(vc), ve)
+        slots = np.array([5, 40, -1], dtype=np.int64)
+        pkv.kv_cache_append(k, v, kc, vc, torch.from_numpy(slots).to(dev))
+        ka, va, nbad = oracle.kv_append(ke, ve, host(k), host(v), slots, B)
+        assert nbad == 0
+        assert np.array_equal(host(kc), ka) and np.array_equal(host(vc), va)
+    finally:
+        pkv.set_debug_checks(before)
+    clean(dev)
