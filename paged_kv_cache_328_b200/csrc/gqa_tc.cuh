@@ -38,9 +38,11 @@
 //   warp 0     producer: the unit's query tile (4-D TMA box, double-buffered) and
 //              the 128-token K/V tiles (2-D TMA boxes per (block, K/V head) run,
 //              128-byte swizzle, kNS stages);
-//   warp 1     allocates / frees the tensor memory; its lane 0 issues every MMA;
+//   warp 1     allocates / frees the tensor memory; its lane 0 issues the S products;
 //   warps 2-9  softmax and epilogue, group (w - 2) / 4; warp w owns tensor-memory
-//              lanes 32*(w%4) ... (tokens of S^T, dimensions of O^T).
+//              lanes 32*(w%4) ... (tokens of S^T, dimensions of O^T);
+//   warp 10    its lane 0 issues the P V products;
+//   warp 11    V producer: the V half of each K/V tile, published by warp 0.
 // P^T of a tile is written over the tile's K slabs (dead once S^T is computed).
 // Each group exchanges reduction partials through shared memory and its own
 // mbarrier (bounded waits: a failing wait cannot strand the other warps).
@@ -51,8 +53,10 @@
 namespace pkv {
 
 constexpr int kKtTile = 128;         // tokens per K/V tile = M of S^T = K of O^T
-constexpr int kKtSoftmaxWarps = 8;   // two groups of four
-constexpr int kKtThreads = (2 + kKtSoftmaxWarps) * 32;
+constexpr int kKtSoftmaxWarps = 8;   // two groups of four: warps 2-9
+constexpr int kKtPvWarp = 2 + kKtSoftmaxWarps;  // issues the P V products
+constexpr int kKtVWarp = 3 + kKtSoftmaxWarps;   // issues the V tiles' TMA loads
+constexpr int kKtThreads = (4 + kKtSoftmaxWarps) * 32;
 constexpr float kKtRescaleLog2 = 8.0f;
 
 // Instruction descriptor for kind::f16 with fp32 accumulation and either operand
@@ -81,12 +85,13 @@ struct KtTraits {
   static constexpr int kQBytes = 2 * kQSlab;
   static constexpr int kQOffset = kNS * kStageBytes;
   static constexpr int kHdrOffset = kQOffset + 2 * kQBytes;  // after two query buffers
-  static constexpr int kRedOffset = kHdrOffset + kNS * 32;   // [group][parity][NH][4 warps] floats
-  static constexpr int kWarpOffset = kRedOffset + 2 * 2 * NH * 4 * 4;  // [softmax warp][mref NH, tmp NH]
-  static constexpr int kVoteOffset = kWarpOffset + kKtSoftmaxWarps * 2 * NH * 4;  // [group][parity][4] ints
+  static constexpr int kRowsOffset = kHdrOffset + kNS * 32;  // [NS][32] pool rows of a tile's runs (-1: none)
+  static constexpr int kRedOffset = kRowsOffset + kNS * 128;  // [group][parity][NH][4 warps] floats
+  static constexpr int kWarpOffset = kRedOffset + 2 * 2 * NH * 4 * 4;  // [softmax warp][mref, tmp, 1/l: NH each]
+  static constexpr int kVoteOffset = kWarpOffset + kKtSoftmaxWarps * 3 * NH * 4;  // [group][parity][4] ints
   static constexpr int kBarOffset = kVoteOffset + 2 * 2 * 4 * 4;
-  // full[NS], empty[NS], q_full[2], q_empty[2], s_full[2], s_free[2], p_full, pv_done, grp[2], drain
-  static constexpr int kNumBars = 2 * kNS + 13;
+  // full[NS], empty[NS], q_full[2], q_empty[2], s_full[2], s_free[2], p_full, pv_done, grp[2], drain[2], meta[NS]
+  static constexpr int kNumBars = 3 * kNS + 14;
   static constexpr int kTmemSlotOffset = kBarOffset + kNumBars * 8;
   static constexpr int kAbortOffset = kTmemSlotOffset + 8;
   static constexpr int kSmemBytes = kAbortOffset + 8;
@@ -123,6 +128,20 @@ __device__ __forceinline__ bool mbar_spin_bounded(uint64_t* bar, uint32_t parity
     if (clock64() - t0 > kWaitLimitCycles) return false;
   }
 }
+
+// Bulk (copy-engine) store of `bytes` contiguous bytes from this CTA's shared
+// memory to global memory, tracked by the issuing thread's bulk async-group.
+// Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_addr(ssrc)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The shared-memory sources of this thread's bulk stores may be overwritten.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// This thread's bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ---- cross-warp reductions of one softmax group ------------------------------
 
@@ -189,6 +208,15 @@ __device__ __forceinline__ bool group_reduce(const float (&v)[N], float* red, fl
   }
   __syncwarp();
   return true;
+}
+
+// Barrier of the group's four warps (same barrier as its reductions).
+__device__ __forceinline__ bool group_sync(uint64_t* grp, int& k, int lane, volatile int* abort_flag) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(grp);
+  const bool ok = __all_sync(0xffffffffu, mbar_spin_bounded(grp, (uint32_t)(k & 1), abort_flag));
+  ++k;
+  return ok;
 }
 
 // OR of one predicate over the group's 128 threads (same barrier as its reductions).
@@ -258,7 +286,9 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
   uint64_t* p_full = q_full + 8;
   uint64_t* pv_done = q_full + 9;
   uint64_t* grp = q_full + 10;       // [2]: one per softmax group
-  uint64_t* drain = q_full + 12;
+  uint64_t* drain = q_full + 12;     // [2]: one per MMA issuer
+  uint64_t* meta = q_full + 14;      // [NS]: a tile's header and pool rows are published
+  int* run_rows = reinterpret_cast<int*>(smem + Tr::kRowsOffset);
   int4* hdr = reinterpret_cast<int4*>(smem + Tr::kHdrOffset);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::kTmemSlotOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Tr::kAbortOffset);
@@ -275,7 +305,8 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
 #pragma unroll
     for (int i = 0; i < NS; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], 3);  // the P V commit, then one arrival per softmax group
+      mbar_init(&meta[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
@@ -286,7 +317,8 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
     }
     mbar_init(p_full, kKtSoftmaxWarps);
     mbar_init(pv_done, 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -402,22 +434,25 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
             flag_error(PKV_DEV_BLOCK_ID);
         }
         const unsigned loads = __ballot_sync(0xffffffffu, load);
+        const int y = load ? (phys * Hkv + cur.kvh) * B + (u_t0 % B) : -1;
+        // publish the tile (header, pool row of each run) for the V producer, arm the
+        // stage's barrier with the bytes of both halves, then load the K half
+        run_rows[stage * 32 + lane] = y;
         if (lane == 0) {
           const int flags = done ? kTileEnd : ((i == 0 ? kTileFirst : 0) | (i == n_tiles - 1 ? kTileLast : 0));
           hdr[2 * stage] = make_int4(cur.s, cur.kvh | (cur.rt << 16), cur.p | (cur.n_parts << 16),
                                      n_valid | (flags << 16));
           hdr[2 * stage + 1] = make_int4(tile_t0, cur.ctx, 0, 0);
-          mbar_arrive_expect_tx(&full[stage], (uint32_t)__popc(loads) * 4u * run_bytes);
         }
         __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[stage], (uint32_t)__popc(loads) * 4u * run_bytes);
+          mbar_arrive(&meta[stage]);
+        }
         if (load) {
-          const int y = (phys * Hkv + cur.kvh) * B + (u_t0 % B);
           unsigned char* kt = smem + stage * Tr::kStageBytes + lane * unit_rows * 128;
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            tma_load_2d(kt + hf * Tr::kSlab, &prm.tmap_k, hf * 64, y, &full[stage], policy);
-            tma_load_2d(kt + (2 + hf) * Tr::kSlab, &prm.tmap_v, hf * 64, y, &full[stage], policy);
-          }
+          for (int hf = 0; hf < 2; ++hf) tma_load_2d(kt + hf * Tr::kSlab, &prm.tmap_k, hf * 64, y, &full[stage], policy);
         }
         if (i == 0 && !done) {
           u_next = __shfl_sync(0xffffffffu, u_next_lane0, 0);
@@ -437,95 +472,121 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
       for (int j = max(0, nu - 2); j < nu; ++j)
         if (!mbar_wait_bounded(&q_full[j & 1], (j >> 1) & 1, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
     }
-  } else if (warp == 1) {
-    // ----------------------------- MMA issuer -----------------------------
-    // Event driven: each pass issues the oldest pending P V product whose P^T is
-    // written, then the next S product whose K/V tile, S buffer (and, opening a
-    // unit, query tile) are ready, so neither waits behind the other.  Shared-
-    // memory descriptors are formed once; an MMA adds a constant offset to the
-    // start-address field (16-byte units; every operand lies below 256 KB).
+  } else if (warp == kKtVWarp) {
+    // ------------------------------ V producer ------------------------------
+    // Follows the K producer tile by tile: once a tile is published (meta), each
+    // run's V rows go to the stage's V slabs, completing on the same barrier.
+    const uint64_t policy = l2_evict_first();
+    const int unit_rows = min(prm.block_size, kKtTile);
+    for (int t = 0;; ++t) {
+      const int stage = t % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&meta[stage], (t / NS) & 1, abort_flag))) {
+        if (lane == 0) {
+          flag_error(PKV_DEV_WAIT_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      if ((hdr[2 * stage].w >> 16) & kTileEnd) break;
+      const int y = run_rows[stage * 32 + lane];
+      if (y >= 0) {
+        unsigned char* vt = smem + stage * Tr::kStageBytes + 2 * Tr::kSlab + lane * unit_rows * 128;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) tma_load_2d(vt + hf * Tr::kSlab, &prm.tmap_v, hf * 64, y, &full[stage], policy);
+      }
+    }
+  } else if (warp == 1 || warp == kKtPvWarp) {
+    // ----------------------------- MMA issuers -----------------------------
+    // Warp 1 issues the S products, warp kKtPvWarp the P V products, each in tile
+    // order with its own commits, so that neither waits behind the other's
+    // issue.  Shared-memory descriptors are formed once; an MMA adds a constant
+    // offset to the start-address field (16-byte units; every operand lies below
+    // 256 KB).
     if (lane == 0) {
-      constexpr uint32_t kIdescS = umma_idesc_ab<T>(kKtTile, NR, false, false);
-      constexpr uint32_t kIdescO = umma_idesc_ab<T>(D, Tr::kPW, true, true);
-      const uint64_t desc_stage0 = umma_desc_sw128(smem_addr(smem), 16, 1024);         // K (A of S), P^T (B of O)
-      const uint64_t desc_v0 = umma_desc_sw128(smem_addr(smem + 2 * Tr::kSlab), Tr::kSlab, 1024);  // V (A of O)
-      const uint64_t desc_p0 = umma_desc_sw128(smem_addr(smem), Tr::kSlab, 1024);
-      const uint64_t desc_q0 = umma_desc_sw128(smem_addr(smem + Tr::kQOffset), 16, 1024);
       bool ok = true;
-      int nq = 0;         // query tiles consumed
-      int ts = 0;         // next tile whose S product is issued
-      int tp = 0;         // next tile whose P V product is issued
-      bool end_seen = false;
-      bool first_of[4] = {false, false, false, false};  // by tile & 3: at most 4 tiles between S and P V
-      long long t_idle = clock64();
-      while (true) {
-        bool progressed = false;
-        if (tp < ts && mbar_test(p_full, (uint32_t)(tp & 1))) {
-          // O^T += V^T [P_hi | P_lo]^T for tile tp (P^T over the tile's K slabs)
+      if (warp == 1) {
+        constexpr uint32_t kIdescS = umma_idesc_ab<T>(kKtTile, NR, false, false);
+        const uint64_t desc_k0 = umma_desc_sw128(smem_addr(smem), 16, 1024);
+        const uint64_t desc_q0 = umma_desc_sw128(smem_addr(smem + Tr::kQOffset), 16, 1024);
+        int nq = 0;  // query tiles consumed
+        for (int t = 0;; ++t) {
+          const int stage = t % NS;
+          if (!mbar_wait_bounded(&full[stage], (t / NS) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int flags = hdr[2 * stage].w >> 16;
+          if (flags & kTileEnd) break;
+          if (flags & kTileFirst) {
+            if (!mbar_wait_bounded(&q_full[nq & 1], (nq >> 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            ++nq;
+          }
+          const int qb = (nq - 1) & 1;
+          const int sb = t & 1;
+          if (t >= 2 && !mbar_wait_bounded(&s_free[sb], ((t >> 1) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const int st = tp % NS;
-          const uint64_t a0 = desc_v0 + (uint64_t)((st * Tr::kStageBytes) >> 4);
-          const uint64_t b0 = desc_p0 + (uint64_t)((st * Tr::kStageBytes) >> 4);
-          const bool fp = first_of[tp & 3];
+          const uint64_t a0 = desc_k0 + (uint64_t)((stage * Tr::kStageBytes) >> 4);
+          const uint64_t b0 = desc_q0 + (uint64_t)((qb * Tr::kQBytes) >> 4);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            // 16 columns = 32 bytes inside a 64-column slab
+            const uint32_t ka = (uint32_t)((k >> 2) * Tr::kSlab + (k & 3) * 32) >> 4;
+            const uint32_t kb = (uint32_t)((k >> 2) * Tr::kQSlab + (k & 3) * 32) >> 4;
+            umma_f16(tmem_base + (uint32_t)(sb * NR), a0 + ka, b0 + kb, kIdescS, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[sb]);
+          if (flags & kTileLast) umma_commit(&q_empty[qb]);
+        }
+      } else {
+        constexpr uint32_t kIdescO = umma_idesc_ab<T>(D, Tr::kPW, true, true);
+        const uint64_t desc_v0 = umma_desc_sw128(smem_addr(smem + 2 * Tr::kSlab), Tr::kSlab, 1024);  // V (A)
+        const uint64_t desc_p0 = umma_desc_sw128(smem_addr(smem), Tr::kSlab, 1024);  // P^T over the K slabs (B)
+        for (int t = 0;; ++t) {
+          const int stage = t % NS;
+          // the stage is released by this warp's commit below, so its header stays valid
+          if (!mbar_wait_bounded(&full[stage], (t / NS) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int flags = hdr[2 * stage].w >> 16;
+          if (flags & kTileEnd) break;
+          if (!mbar_wait_bounded(p_full, (uint32_t)(t & 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a0 = desc_v0 + (uint64_t)((stage * Tr::kStageBytes) >> 4);
+          const uint64_t b0 = desc_p0 + (uint64_t)((stage * Tr::kStageBytes) >> 4);
+          const bool fp = flags & kTileFirst;
 #pragma unroll
           for (int k = 0; k < kKtTile / 16; ++k)  // 16 tokens per step: 16 rows x 128 bytes
             umma_f16(tmem_base + Tr::kOCol, a0 + (uint64_t)(k * (2048 >> 4)), b0 + (uint64_t)(k * (2048 >> 4)),
                      kIdescO, (fp && k == 0) ? 0u : 1u);
-          umma_commit(&empty[st]);
+          umma_commit(&empty[stage]);
           umma_commit(pv_done);
-          ++tp;
-          progressed = true;
-        }
-        if (!end_seen) {
-          const int stage = ts % NS;
-          if (mbar_test(&full[stage], (uint32_t)((ts / NS) & 1))) {
-            const int flags = hdr[2 * stage].w >> 16;
-            if (flags & kTileEnd) {
-              end_seen = true;
-              progressed = true;
-            } else {
-              const bool first = flags & kTileFirst;
-              const int sb = ts & 1;
-              const bool q_ok = !first || mbar_test(&q_full[nq & 1], (uint32_t)((nq >> 1) & 1));
-              const bool s_ok = ts < 2 || mbar_test(&s_free[sb], (uint32_t)(((ts >> 1) - 1) & 1));
-              if (q_ok && s_ok) {
-                if (first) ++nq;
-                const int qb = (nq - 1) & 1;
-                tc_fence_after();
-                const uint64_t a0 = desc_stage0 + (uint64_t)((stage * Tr::kStageBytes) >> 4);
-                const uint64_t b0 = desc_q0 + (uint64_t)((qb * Tr::kQBytes) >> 4);
-#pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
-                  // 16 columns = 32 bytes inside a 64-column slab
-                  const uint32_t ka = (uint32_t)((k >> 2) * Tr::kSlab + (k & 3) * 32) >> 4;
-                  const uint32_t kb = (uint32_t)((k >> 2) * Tr::kQSlab + (k & 3) * 32) >> 4;
-                  umma_f16(tmem_base + (uint32_t)(sb * NR), a0 + ka, b0 + kb, kIdescS, k > 0 ? 1u : 0u);
-                }
-                umma_commit(&s_full[sb]);
-                if (flags & kTileLast) umma_commit(&q_empty[qb]);
-                first_of[ts & 3] = first;
-                ++ts;
-                progressed = true;
-              }
-            }
+          // a unit's last stage also holds its output rows until they are stored:
+          // there each softmax group releases it; elsewhere this thread does
+          if (!(flags & kTileLast)) {
+            mbar_arrive(&empty[stage]);
+            mbar_arrive(&empty[stage]);
           }
-        }
-        if (end_seen && tp == ts) break;
-        if (progressed) {
-          t_idle = clock64();
-        } else if (*abort_flag || clock64() - t_idle > kWaitLimitCycles) {
-          ok = false;
-          break;
         }
       }
       if (!ok) {
         flag_error(PKV_DEV_WAIT_TIMEOUT);
         *abort_flag = 1;
       }
-      // every MMA issued above must be complete before the tensor memory is freed
-      umma_commit(drain);
+      // every MMA this thread issued must be complete before the tensor memory is freed
+      uint64_t* my_drain = warp == 1 ? drain : drain + 1;
+      umma_commit(my_drain);
       int no_abort = 0;
-      if (!mbar_wait_bounded(drain, 0, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
+      if (!mbar_wait_bounded(my_drain, 0, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
     }
     __syncwarp();
   } else {
@@ -542,8 +603,9 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
     uint64_t* my_grp = &grp[sg];
     // this warp's copies of its rows' reference maxima and of a per-row scratch
     // (the excess of a tile's maxima over the references, then the row sums)
-    float* mref = reinterpret_cast<float*>(smem + Tr::kWarpOffset) + (warp - 2) * 2 * NH;
+    float* mref = reinterpret_cast<float*>(smem + Tr::kWarpOffset) + (warp - 2) * 3 * NH;
     float* tmp = mref + NH;
+    float* inv = tmp + NH;
     const float4* mref4 = reinterpret_cast<const float4*>(mref);
     const float4* tmp4 = reinterpret_cast<const float4*>(tmp);
     float lpart[NH];  // this thread's share of each row's sum of weights
@@ -752,7 +814,7 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
 
       if (flags & kTileLast) {
         // epilogue: the unit's products are complete once P V of this tile is;
-        // tmp = the group's row sums of weights
+        // tmp = the group's row sums of weights, inv = their reciprocals
         if (!wait_pv(j)) {
           failed = true;
           break;
@@ -761,11 +823,17 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
           failed = true;
           break;
         }
+        if (lane < NH) inv[lane] = tmp[lane] > 0.f ? 1.f / tmp[lane] : 0.f;
+        __syncwarp();
         tc_fence_after();
         const int us = hd.x, ukv = hd.y & 0xffff, up = hd.z & 0xffff, un = hd.z >> 16;
         const int rows = min(Tq, Lq - rt * Tq) * G;  // real rows of this tile
         const size_t row0 = (size_t)us * Lq + (size_t)rt * Tq;  // (sequence, first query token)
-        int tq_local = r0 / G, g = r0 - (r0 / G) * G;
+        // The group's output rows go through the tile's V slabs (dead once P V is
+        // complete; the stage stays held until the rows are stored): thread tl
+        // writes dimension tl of each row, then one thread stores the rows with the
+        // copy engine, so no warp waits on scattered global stores.
+        float* stg = reinterpret_cast<float*>(smem + stage * Tr::kStageBytes + 2 * Tr::kSlab) + sg * NH * D;
 #pragma unroll
         for (int c = 0; c < NH / 8; ++c) {
           uint32_t vh[8], vl[8];
@@ -777,26 +845,45 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int r = 8 * c + i;  // row r0 + r
-            if (r0 + r < rows) {
-              const size_t sh = (row0 + tq_local) * prm.num_heads + (size_t)ukv * G + g;
-              const float v = __uint_as_float(vh[i]) + __uint_as_float(vl[i]);
-              const float l = tmp[r];
-              if (un == 1) {
-                prm.out[sh * D + tl] = l > 0.f ? v * (1.f / l) : 0.f;
-              } else {
-                prm.ws_acc[(sh * prm.max_parts + up) * D + tl] = v;
-                if (tl == r) prm.ws_ml[sh * prm.max_parts + up] = make_float2(mref[r], l);
-              }
-            }
-            if (++g == G) {
-              g = 0;
-              ++tq_local;
-            }
+            const float v = __uint_as_float(vh[i]) + __uint_as_float(vl[i]);
+            stg[r * D + tl] = un == 1 ? v * inv[r] : v;
           }
         }
+        if (un != 1 && tl < NH && r0 + tl < rows) {
+          const int R = r0 + tl;
+          const size_t sh = (row0 + R / G) * prm.num_heads + (size_t)ukv * G + R % G;
+          prm.ws_ml[sh * prm.max_parts + up] = make_float2(mref[tl], tmp[tl]);
+        }
+        fence_proxy_async_smem();  // the staged rows are read by the copy engine
         tc_fence_before();
+        if (!group_sync(my_grp, gk, lane, abort_flag)) {
+          failed = true;
+          break;
+        }
+        if (warp == 2 + 4 * sg && lane == 0) {
+          const int r_end = min(r0 + NH, rows);
+          if (un == 1) {
+            // runs of rows of one query token are consecutive query heads
+            for (int R = r0; R < r_end;) {
+              const int tq = R / G, g = R - tq * G;
+              const int run = min(r_end - R, G - g);
+              bulk_store(prm.out + ((row0 + tq) * prm.num_heads + (size_t)ukv * G + g) * D, stg + (R - r0) * D,
+                         (uint32_t)(run * D * 4));
+              R += run;
+            }
+          } else {
+            for (int R = r0; R < r_end; ++R) {
+              const size_t sh = (row0 + R / G) * prm.num_heads + (size_t)ukv * G + R % G;
+              bulk_store(prm.ws_acc + (sh * prm.max_parts + up) * D, stg + (R - r0) * D, (uint32_t)(D * 4));
+            }
+          }
+          bulk_commit();
+          bulk_wait_read();
+          mbar_arrive(&empty[stage]);
+        }
       }
     }
+    bulk_wait_all();  // this thread's output stores are complete
     if (failed && lane == 0) {
       flag_error(PKV_DEV_WAIT_TIMEOUT);
       *abort_flag = 1;

@@ -295,9 +295,13 @@ bool use_gqa_kernel(int Hq, int Hkv, int B, int NB, pkv_dtype dt) {
 //  * kTc128: the row-major tcgen05 kernel (multi_query_tc.cuh) above that (or
 //    head_dim 64 above 16 rows): 128-row tiles of floor(128 / G) whole query tokens;
 //  * kMmaSync: the warp-level kernel (decode_gqa.cuh), 16-row tiles.
+// Measured on B200 (batch-256 layer, 8 K/V heads x 128, bf16, attention call): the
+// token-major kernel is ahead from 8 rows (G = 8: 5.56 vs 5.49 TB/s; G = 16: 5.52
+// vs 4.94; 16 rows of a 4-token verify: 5.47 vs 4.94) and behind below (G = 2:
+// 5.48 vs 5.87; G = 4: 5.48 vs 5.79).
 // The choice depends only on the shapes, so the workspace query and the launch agree.
 enum class TcPath { kMmaSync, kKt, kTc128 };
-constexpr long long kKtMinRows = 16;
+constexpr long long kKtMinRows = 7;
 constexpr long long kKtMaxRows = 64;
 
 TcPath tc_path(long long q_len, int group, int head_dim) {
