@@ -564,10 +564,15 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
           const uint64_t a0 = desc_v0 + (uint64_t)((stage * Tr::kStageBytes) >> 4);
           const uint64_t b0 = desc_p0 + (uint64_t)((stage * Tr::kStageBytes) >> 4);
           const bool fp = flags & kTileFirst;
+          // 16 tokens per step (16 rows x 128 bytes); steps wholly past the tile's
+          // valid tokens add nothing (their weights are 0) and are skipped; an
+          // empty tile still runs one step (zero weights) so that O starts at 0
+          const int steps = max(1, ((hdr[2 * stage].w & 0xffff) + 15) / 16);
 #pragma unroll
-          for (int k = 0; k < kKtTile / 16; ++k)  // 16 tokens per step: 16 rows x 128 bytes
-            umma_f16(tmem_base + Tr::kOCol, a0 + (uint64_t)(k * (2048 >> 4)), b0 + (uint64_t)(k * (2048 >> 4)),
-                     kIdescO, (fp && k == 0) ? 0u : 1u);
+          for (int k = 0; k < kKtTile / 16; ++k)
+            if (k < steps)
+              umma_f16(tmem_base + Tr::kOCol, a0 + (uint64_t)(k * (2048 >> 4)), b0 + (uint64_t)(k * (2048 >> 4)),
+                       kIdescO, (fp && k == 0) ? 0u : 1u);
           umma_commit(&empty[stage]);
           umma_commit(pv_done);
           // a unit's last stage also holds its output rows until they are stored:
@@ -789,10 +794,13 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
         }
       }
       // V rows past the tile's valid tokens may hold anything (NaN in unwritten
-      // slots, stale rows of earlier tiles): zero them so that 0 * V stays 0
-      if (n_valid < kKtTile) {
+      // slots, stale rows of earlier tiles): zero those that the P V product
+      // reads (up to the 16-token step holding the last valid token; an empty
+      // tile's one step) so that 0 * V stays 0
+      const int v_end = max(16, (n_valid + 15) / 16 * 16);
+      if (n_valid < v_end) {
         unsigned char* vt = smem + stage * Tr::kStageBytes + 2 * Tr::kSlab;
-        const int per_slab = (kKtTile - n_valid) * 8;
+        const int per_slab = (v_end - n_valid) * 8;
         for (int i = sg * 128 + tl; i < 2 * per_slab; i += 256) {
           const int hf = i / per_slab;
           const int rem = i - hf * per_slab;
@@ -813,18 +821,19 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
       if (lane == 0) mbar_arrive(p_full);
 
       if (flags & kTileLast) {
-        // epilogue: the unit's products are complete once P V of this tile is;
-        // tmp = the group's row sums of weights, inv = their reciprocals
-        if (!wait_pv(j)) {
-          failed = true;
-          break;
-        }
+        // epilogue: tmp = the group's row sums of weights (final once this tile's P
+        // is written, so reduced while its P V product runs), inv = their
+        // reciprocals; then O is complete once P V of this tile is
         if (!group_reduce<NH, false>(lpart, red, tmp, my_grp, gk, q4, lane, abort_flag)) {
           failed = true;
           break;
         }
         if (lane < NH) inv[lane] = tmp[lane] > 0.f ? 1.f / tmp[lane] : 0.f;
         __syncwarp();
+        if (!wait_pv(j)) {
+          failed = true;
+          break;
+        }
         tc_fence_after();
         const int us = hd.x, ukv = hd.y & 0xffff, up = hd.z & 0xffff, un = hd.z >> 16;
         const int rows = min(Tq, Lq - rt * Tq) * G;  // real rows of this tile
