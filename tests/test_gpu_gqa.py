@@ -1,8 +1,9 @@
 """GPU parity of grouped-query paged decode (paged_attn_decode_gqa through the C ABI).
 
-Query head h reads K/V head h // G.  16-bit K/V with 2 <= G <= 16 runs on the
-warp-level tensor-core kernel, 16 < G <= 128 on the tcgen05 kernel (one 128-row
-tile per (sequence, K/V head)); fp32 K/V and G = 1 run on the CUDA-core kernel.
+Query head h reads K/V head h // G.  16-bit K/V with G < 8 runs on the warp-level
+tensor-core kernel, 8 <= G <= 64 (head_dim 128) on the token-major tcgen05 kernel,
+more on the 128-row tcgen05 kernel (head_dim 64 above 16 as well); fp32 K/V and
+G = 1 run on the CUDA-core kernel.
 Tolerances as for multi-head decode: 2e-3 (fp16/bf16), 1e-5 (fp32).
 """
 

@@ -1,5 +1,7 @@
-"""GPU parity of the tcgen05 multi-query kernel (more than 16 query rows per K/V head:
-Lq * G > 16) against the CPU oracle, through the C ABI.
+"""GPU parity of the tcgen05 multi-query kernels (more than 16 query rows per K/V head:
+Lq * G > 16) against the CPU oracle, through the C ABI: with head_dim 128 up to 64
+rows run on the token-major kernel, more on the 128-row kernel; head_dim 64 always
+on the 128-row kernel.
 
 Covers query rows spanning several 128-row tiles (Lq * G > 128), groups that do not
 divide 128 (padding rows in every tile), contexts shorter than Lq (query rows that
