@@ -78,13 +78,16 @@ struct KtTraits {
   static constexpr int NH = NR / 2;                    // rows per softmax group
   // P^T row: hi at column 0, lo at column kPW / 2; kPW / 64 slabs of 128 rows
   static constexpr int kPW = NR <= 32 ? 64 : 2 * NR;
-  static constexpr int kNS = NR <= 32 ? 3 : 2;         // K/V stages of 64 KB
+  static constexpr int kNS = 3;                        // K/V stages of 64 KB
+  // query tiles: two (the next unit's loads while this one runs), one at 64 rows
+  // (shared memory), loaded as soon as the previous unit's last S product is done
+  static constexpr int kNQ = NR <= 32 ? 2 : 1;
   static constexpr int kSlab = kKtTile * 128;          // 128 rows x 64 columns, 16-bit: 16 KB
   static constexpr int kStageBytes = 4 * kSlab;        // K (2 slabs), V (2 slabs)
   static constexpr int kQSlab = NR * 128;
   static constexpr int kQBytes = 2 * kQSlab;
   static constexpr int kQOffset = kNS * kStageBytes;
-  static constexpr int kHdrOffset = kQOffset + 2 * kQBytes;  // after two query buffers
+  static constexpr int kHdrOffset = kQOffset + kNQ * kQBytes;  // after the query buffers
   static constexpr int kRowsOffset = kHdrOffset + kNS * 32;  // [NS][32] pool rows of a tile's runs (-1: none)
   static constexpr int kRedOffset = kRowsOffset + kNS * 128;  // [group][parity][NH][4 warps] floats
   static constexpr int kWarpOffset = kRedOffset + 2 * 2 * NH * 4 * 4;  // [softmax warp][mref, tmp, 1/l: NH each]
@@ -274,6 +277,7 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
   constexpr int D = Tr::D;
   constexpr int NS = Tr::kNS;
   constexpr int NH = Tr::NH;
+  constexpr int NQ = Tr::kNQ;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::kBarOffset);
@@ -323,7 +327,7 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
     fence_mbar_init();
   }
   // query rows that no TMA box covers read as zero (their logits are masked in any case)
-  for (int i = threadIdx.x; i < 2 * Tr::kQBytes / 16; i += blockDim.x)
+  for (int i = threadIdx.x; i < Tr::kNQ * Tr::kQBytes / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(smem + Tr::kQOffset)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (warp == 1) {
@@ -372,8 +376,36 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
 
     int u = (int)blockIdx.x;
     TcUnit cur = describe(u, entry(u));
-    int it = 0;  // tiles issued
-    int nu = 0;  // query tiles issued
+    int it = 0;        // tiles issued
+    // Query tiles (lane 0's bookkeeping): unit n's goes to buffer n % NQ once the S
+    // products of unit n - NQ are done.  A unit's tile is owed from the unit's
+    // start and issued as soon as its buffer is free, also while this warp waits
+    // for a stage, so the K/V tiles never wait for it.
+    int nu = 0;        // query tiles issued
+    int owed = 0;      // units begun (query tiles owed up to this count)
+    TcUnit q_unit = cur;
+    auto q_ready = [&]() {
+      return nu < NQ || mbar_test(&q_empty[nu % NQ], (uint32_t)(((nu / NQ) - 1) & 1));
+    };
+    auto q_issue = [&]() {  // lane 0
+      const int qb = nu % NQ;
+      mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+        tma_load_4d(smem + Tr::kQOffset + qb * Tr::kQBytes + hf * Tr::kQSlab, &prm.tmap_q, hf * 64,
+                    q_unit.kvh * G, q_unit.rt * Tq, q_unit.s, &q_full[qb], policy);
+      ++nu;
+    };
+    // lane 0: wait (bounded) until the owed query tile can be issued, and issue it
+    auto q_settle = [&]() {
+      if (nu == owed) return true;
+      const long long t0 = clock64();
+      while (!q_ready()) {
+        if (*abort_flag || clock64() - t0 > kWaitLimitCycles) return false;
+      }
+      q_issue();
+      return true;
+    };
     bool stop = false;
     while (!stop) {
       const bool done = (long long)u >= total_units;
@@ -381,10 +413,16 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
       int u_next = 0;
       uint2 e_next = make_uint2(0u, 0u);
       if (!done) {
-        // query buffer nu & 1 was last read by the S products of unit nu - 2
-        const int qb = nu & 1;
+        // one query tile owed at a time: the previous unit's is issued first
         int ok = 1;
-        if (nu >= 2 && lane == 0) ok = mbar_wait_bounded(&q_empty[qb], ((nu >> 1) - 1) & 1, abort_flag);
+        if (lane == 0) {
+          ok = q_settle();
+          if (ok) {
+            q_unit = cur;
+            ++owed;
+            if (q_ready()) q_issue();
+          }
+        }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) {
           if (lane == 0) {
@@ -393,14 +431,6 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
           }
           break;
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&q_full[qb], q_bytes);
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_4d(smem + Tr::kQOffset + qb * Tr::kQBytes + hf * Tr::kQSlab, &prm.tmap_q, hf * 64,
-                        cur.kvh * G, cur.rt * Tq, cur.s, &q_full[qb], policy);
-        }
-        ++nu;
       }
       const int n_tok = max(0, cur.t_end - cur.t_begin);
       const int n_tiles = done ? 1 : max(1, (n_tok + kKtTile - 1) / kKtTile);
@@ -414,7 +444,22 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
         const int phys = mine ? __ldg(table + u_t0 / B) : -1;  // u_t0 < ctx <= max_blocks * B
         if (it >= NS) {
           int ok = 1;
-          if (lane == 0) ok = mbar_wait_bounded(&empty[stage], ((it / NS) - 1) & 1, abort_flag);
+          if (lane == 0) {
+            const uint32_t par = ((it / NS) - 1) & 1;
+            if (nu == owed) {
+              ok = mbar_wait_bounded(&empty[stage], par, abort_flag);
+            } else {
+              // poll: the owed query tile goes out as soon as its buffer is free
+              const long long t0 = clock64();
+              while (!mbar_test(&empty[stage], par)) {
+                if (nu < owed && q_ready()) q_issue();
+                if (*abort_flag || clock64() - t0 > kWaitLimitCycles) {
+                  ok = 0;
+                  break;
+                }
+              }
+            }
+          }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) {
             if (lane == 0) {
@@ -463,14 +508,19 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
       u = u_next;
       cur = describe(u, e_next);
     }
+    // the last unit's query tile, if still owed
+    if (lane == 0 && !stop && !q_settle()) {
+      flag_error(PKV_DEV_WAIT_TIMEOUT);
+      *abort_flag = 1;
+    }
     pdl_launch_dependents();
     // never leave with copies in flight into this CTA's shared memory
     if (lane == 0) {
       int no_abort = 0;
       for (int j = max(0, it - NS); j < it; ++j)
         if (!mbar_wait_bounded(&full[j % NS], (j / NS) & 1, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
-      for (int j = max(0, nu - 2); j < nu; ++j)
-        if (!mbar_wait_bounded(&q_full[j & 1], (j >> 1) & 1, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
+      for (int j = max(0, nu - NQ); j < nu; ++j)
+        if (!mbar_wait_bounded(&q_full[j % NQ], (j / NQ) & 1, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
     }
   } else if (warp == kKtVWarp) {
     // ------------------------------ V producer ------------------------------
@@ -518,13 +568,13 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
           const int flags = hdr[2 * stage].w >> 16;
           if (flags & kTileEnd) break;
           if (flags & kTileFirst) {
-            if (!mbar_wait_bounded(&q_full[nq & 1], (nq >> 1) & 1, abort_flag)) {
+            if (!mbar_wait_bounded(&q_full[nq % NQ], (nq / NQ) & 1, abort_flag)) {
               ok = false;
               break;
             }
             ++nq;
           }
-          const int qb = (nq - 1) & 1;
+          const int qb = (nq - 1) % NQ;
           const int sb = t & 1;
           if (t >= 2 && !mbar_wait_bounded(&s_free[sb], ((t >> 1) - 1) & 1, abort_flag)) {
             ok = false;
