@@ -55,6 +55,8 @@ def parse():
                     help="split-context partition size (default: the workload's, else the library's choice)")
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every call from Python in the timed loop instead of replaying CUDA graphs")
     ap.add_argument("--no-targets", action="store_true",
                     help="default workload only: skip timing the long-context layer after it")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline time budget")
@@ -367,11 +369,26 @@ class Step:
             dec_events[1].record(self.stream)
 
 
-def time_steps(step, steps, warmup, pkv, dev, local_rank, world, dist):
+def graph_chunk(steps):
+    """Steps per captured graph: a divisor of the step count, so that the timed
+    replays run exactly `steps` steps."""
+    for m in (10, 8, 5, 4, 2):
+        if steps % m == 0 and steps // m >= 3:
+            return m
+    return 1
+
+
+def time_steps(step, steps, warmup, pkv, dev, local_rank, world, dist, eager=False):
     """W untimed steps, then K timed steps bracketed by a barrier and a synchronize
     on both sides, with the SM clocks sampled during the timed region.  Returns the
     total, per-step and per-attention-call times (CUDA events on the launching
-    stream; the total is the max over ranks) and the clock summary."""
+    stream; the total is the max over ranks) and the clock summary.
+
+    By default the steps run as CUDA graphs (the way a serving loop replays its
+    decode step): M steps are captured once through the public API and replayed
+    K / M times, with an event between replays; the attention call alone is timed
+    the same way from a graph of M calls.  `eager` launches every call from Python
+    instead, so the host's launch cost can show in the device timeline."""
     import torch
     stream = step.stream
 
@@ -385,24 +402,53 @@ def time_steps(step, steps, warmup, pkv, dev, local_rank, world, dist):
     code, reason = pkv.get_device_error(dev)
     if code != 0:
         raise RuntimeError(f"device error word after warm-up: {code} reason {reason}")
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    m = 1 if eager else graph_chunk(steps)
+    if not eager:
+        g_step, g_call = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step):
+            for _ in range(m):
+                step()
+        with torch.cuda.graph(g_call):
+            for _ in range(m):
+                step.attend(step.w.q, step.ix["bt"], step.ix["ctx"], step.out)
+        for _ in range(2):
+            g_step.replay()
+            g_call.replay()
+        torch.cuda.synchronize()
+        run_steps = g_step.replay
     clocks = ClockSampler(local_rank)
     time.sleep(0.3)
-    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    ev = [(mk(), mk(), mk()) for _ in range(steps)]     # step start, attention start / end
-    t_end = mk()
+    n = steps // m
+    ev = [mk() for _ in range(n + 1)]
+    dec = [(mk(), mk()) for _ in range(n)] if eager else None
     barrier()
     torch.cuda.synchronize()
     clocks.mark(True)
-    for i in range(steps):
-        ev[i][0].record(stream)
-        step((ev[i][1], ev[i][2]))
-    t_end.record(stream)
+    ev[0].record(stream)
+    for i in range(n):
+        if eager:
+            step(dec[i])
+        else:
+            run_steps()
+        ev[i + 1].record(stream)
     torch.cuda.synchronize()
     clocks.mark(False)
     barrier()
-    total = ev[0][0].elapsed_time(t_end)
-    per_step = [ev[i][0].elapsed_time(ev[i + 1][0] if i + 1 < steps else t_end) for i in range(steps)]
-    per_call = [e[1].elapsed_time(e[2]) for e in ev]
+    total = ev[0].elapsed_time(ev[n])
+    per_step = [ev[i].elapsed_time(ev[i + 1]) / m for i in range(n)]
+    if eager:
+        per_call = [e0.elapsed_time(e1) for e0, e1 in dec]
+    else:
+        # the attention call alone, from the graph of m calls
+        cev = [mk() for _ in range(n + 1)]
+        cev[0].record(stream)
+        for i in range(n):
+            g_call.replay()
+            cev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        per_call = [cev[i].elapsed_time(cev[i + 1]) / m for i in range(n)]
+        del g_step, g_call
     dec_mean = statistics.mean(per_call)
     if world > 1:
         total, dec_mean = max_over_ranks([total, dec_mean], dist, dev)
@@ -410,7 +456,10 @@ def time_steps(step, steps, warmup, pkv, dev, local_rank, world, dist):
     if code != 0:
         raise RuntimeError(f"device error word after the timed steps: {code} reason {reason}")
     return dict(total_ms=total, step=spread(per_step), call=spread(per_call), call_mean=dec_mean,
-                clocks=clocks.summary())
+                clocks=clocks.summary(),
+                timing=("eager: every call launched from Python" if eager else
+                        f"CUDA graphs of {m} steps (and of {m} attention calls) captured through the public "
+                        f"API, replayed {n} times with an event between replays"))
 
 
 def roofline(kind, kv_bytes, call_ms, peak, peak_src, traffic, call):
@@ -471,7 +520,7 @@ def run_gpu(a, rank, world, local_rank):
         tuned = {str(k): round(v, 5) for k, v in times.items()}
     step = Step(pkv, w, Lq, pt, ix, dev)
     stream = step.stream
-    t = time_steps(step, a.steps, a.warmup, pkv, dev, local_rank, world, dist)
+    t = time_steps(step, a.steps, a.warmup, pkv, dev, local_rank, world, dist, eager=a.eager)
     ms = t["total_ms"]
     dec_ms = t["call_mean"]
     out = step.out
@@ -582,6 +631,7 @@ def run_gpu(a, rank, world, local_rank):
             "l2": f"no flush: K/V pool {w.k_pool.numel() * w.k_pool.element_size() * 2 / 1e9:.2f} GB "
                   f"= {w.k_pool.numel() * w.k_pool.element_size() * 2 / 126e6:.0f}x L2",
             "parallelism": f"replicas x{world}",
+            "timing": t["timing"],
         },
         "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
         "pct_of_hbm_peak_basis": "MEASURED_PEAKS.json hbm_gbs: a device-to-device copy counting read + write "
@@ -623,7 +673,7 @@ def run_gpu(a, rank, world, local_rank):
         w2 = wl.make_longctx(device=dev)
         ix2 = prepare(w2, 1, dev)
         step2 = Step(pkv, w2, 1, w2.partition_tokens, ix2, dev)
-        t2 = time_steps(step2, a.steps, a.warmup, pkv, dev, local_rank, world, dist)
+        t2 = time_steps(step2, a.steps, a.warmup, pkv, dev, local_rank, world, dist, eager=a.eager)
         kv2 = w2.kv_bytes_attended()
         ms2 = t2["total_ms"] / a.steps
         v2, _ = job_throughput(kv2, [ms2] * world)

@@ -117,19 +117,25 @@ __device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontro
 
 // ---------------------------------------------------------------------------
 // 1. plan (one CTA).  With `sort`, one warp orders the units by decreasing
-//    length in 256-token buckets with a stable counting sort: within a bucket
+//    length (unit_bucket) with a stable counting sort: within a bucket
 //    the units keep sequence order, so sequences that share prefix blocks stay
 //    adjacent and their shared blocks are re-read from L2.  Longest-first lets
 //    the dynamically scheduled CTAs end together.
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 128;
-constexpr int kPlanBucketShift = 8;  // 256 tokens per bucket
 constexpr int kPlanSortMaxSeqs = 4096;  // sorted lists: num_seqs * partitions <= this
 static_assert(kPlanBuckets % 32 == 0, "the bucket scan gives every lane the same number of buckets");
 
+// Sort key of a unit of len tokens, non-decreasing in len: 8-token buckets up to
+// 512 tokens, 256-token buckets above (the last bucket takes everything past
+// 16.4K).  The units claimed last decide how evenly the CTAs end and they are
+// the shortest, so the short end is sorted finely (a unit of 250 tokens holds a
+// CTA ~6 us); above it the wide buckets keep sequences of similar length in
+// submission order, so that samples sharing prefix blocks run side by side.
 __device__ __forceinline__ int unit_bucket(int len) {
-  return min(kPlanBuckets - 1, (len + (1 << kPlanBucketShift) - 1) >> kPlanBucketShift);
+  if (len <= 512) return (len + 7) >> 3;                                  // 0 .. 64
+  return min(kPlanBuckets - 1, 64 + ((len - 512 + 255) >> 8));            // 65 .. 127
 }
 
 __global__ void __launch_bounds__(kPlanThreads)
