@@ -386,8 +386,9 @@ def time_steps(step, steps, warmup, pkv, dev, local_rank, world, dist, eager=Fal
 
     By default the steps run as CUDA graphs (the way a serving loop replays its
     decode step): M steps are captured once through the public API and replayed
-    K / M times, with an event between replays; the attention call alone is timed
-    the same way from a graph of M calls.  `eager` launches every call from Python
+    K / M times, each replay between two events; a graph of M attention calls is
+    replayed after each of them (outside the steps' events), so that both see the
+    same clocks under the power cap.  `eager` launches every call from Python
     instead, so the host's launch cost can show in the device timeline."""
     import torch
     stream = step.stream
@@ -420,34 +421,29 @@ def time_steps(step, steps, warmup, pkv, dev, local_rank, world, dist, eager=Fal
     clocks = ClockSampler(local_rank)
     time.sleep(0.3)
     n = steps // m
-    ev = [mk() for _ in range(n + 1)]
-    dec = [(mk(), mk()) for _ in range(n)] if eager else None
+    ev = [(mk(), mk()) for _ in range(n)]       # around each step replay (or eager step)
+    dec = [(mk(), mk()) for _ in range(n)]      # around each attention-call replay (or eager call)
     barrier()
     torch.cuda.synchronize()
     clocks.mark(True)
-    ev[0].record(stream)
     for i in range(n):
+        ev[i][0].record(stream)
         if eager:
             step(dec[i])
         else:
             run_steps()
-        ev[i + 1].record(stream)
+        ev[i][1].record(stream)
+        if not eager:
+            dec[i][0].record(stream)
+            g_call.replay()
+            dec[i][1].record(stream)
     torch.cuda.synchronize()
     clocks.mark(False)
     barrier()
-    total = ev[0].elapsed_time(ev[n])
-    per_step = [ev[i].elapsed_time(ev[i + 1]) / m for i in range(n)]
-    if eager:
-        per_call = [e0.elapsed_time(e1) for e0, e1 in dec]
-    else:
-        # the attention call alone, from the graph of m calls
-        cev = [mk() for _ in range(n + 1)]
-        cev[0].record(stream)
-        for i in range(n):
-            g_call.replay()
-            cev[i + 1].record(stream)
-        torch.cuda.synchronize()
-        per_call = [cev[i].elapsed_time(cev[i + 1]) / m for i in range(n)]
+    per_step = [e0.elapsed_time(e1) / m for e0, e1 in ev]
+    per_call = [e0.elapsed_time(e1) / m for e0, e1 in dec]
+    total = sum(per_step) * m  # the K steps' device time
+    if not eager:
         del g_step, g_call
     dec_mean = statistics.mean(per_call)
     if world > 1:
