@@ -116,16 +116,19 @@ __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepc
 __device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
-// 1. plan (one CTA).  With `sort`, one warp orders the units by decreasing
-//    length (unit_bucket) with a stable counting sort: within a bucket
-//    the units keep sequence order, so sequences that share prefix blocks stay
+// 1. plan (one CTA).  With `sort`, the units are ordered by decreasing length
+//    (unit_bucket) with a stable counting sort: within a bucket the units keep
+//    (sequence, partition) order, so sequences that share prefix blocks stay
 //    adjacent and their shared blocks are re-read from L2.  Longest-first lets
-//    the dynamically scheduled CTAs end together.
+//    the dynamically scheduled CTAs end together.  Up to kPlanThreads sequences
+//    are placed in one pass, one thread per sequence; longer lists take one warp
+//    over runs of 32 sequences.
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 128;
 constexpr int kPlanSortMaxSeqs = 4096;  // sorted lists: num_seqs * partitions <= this
 static_assert(kPlanBuckets % 32 == 0, "the bucket scan gives every lane the same number of buckets");
+static_assert(kPlanThreads == 1024 && kPlanBuckets == 128, "one-pass sort: 32 warps, eight threads per key");
 
 // Sort key of a unit of len tokens, non-decreasing in len: 8-token buckets up to
 // 512 tokens, 256-token buckets above (the last bucket takes everything past
@@ -138,10 +141,135 @@ __device__ __forceinline__ int unit_bucket(int len) {
   return min(kPlanBuckets - 1, 64 + ((len - 512 + 255) >> 8));            // 65 .. 127
 }
 
+// One pass of the stable counting sort with one thread per sequence (num_seqs <=
+// kPlanThreads).  A sequence's partitions but the last are full (bucket
+// key_full); its last partition has bucket key.  Bucket key_full holds its units
+// in (sequence, partition) order: unit (s, p) sits after every unit of the
+// sequences before s in that bucket (an exclusive scan over the sequences).
+// Any other bucket holds last partitions only, in sequence order: the rank of s
+// among the sequences with its key is its rank within its warp (match_any)
+// plus the count of that key in the warps before (a scan over the 32 warps).
+__device__ __forceinline__ void plan_sort_one_pass(const int32_t* __restrict__ context_lens, int num_seqs,
+                                                   int max_ctx, int part_tokens, uint2* __restrict__ units,
+                                                   int* __restrict__ counters) {
+  constexpr int kWarps = kPlanThreads / 32;
+  __shared__ int cnt[kWarps][kPlanBuckets];  // per warp and key: count, then exclusive offset
+  __shared__ int total[kPlanBuckets];        // sequences whose last partition has key k
+  __shared__ int start[kPlanBuckets];        // first position of bucket k
+  __shared__ int wsum[kWarps];               // per warp: units in bucket key_full, then exclusive prefix
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int s = tid;
+  const bool live = s < num_seqs;
+  int ctx = 0;
+  if (live) {
+    const int raw = context_lens[s];
+    if (raw < 0 || raw > max_ctx) flag_error(PKV_DEV_CONTEXT_LEN);
+    ctx = clamp_ctx(raw, max_ctx);
+  }
+  const int n = live ? parts_of(ctx, part_tokens) : 0;
+  const int nfull = max(n - 1, 0);
+  const int key_full = unit_bucket(part_tokens);
+  const int key = live ? unit_bucket(ctx - (n - 1) * part_tokens) : -1;
+  for (int i = tid; i < kWarps * kPlanBuckets; i += kPlanThreads) (&cnt[0][0])[i] = 0;
+  // this sequence's units in bucket key_full, scanned over the warp
+  const int gv = nfull + (key == key_full ? 1 : 0);
+  int g_incl = gv;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, g_incl, o);
+    if (lane >= o) g_incl += v;
+  }
+  const unsigned same = __match_any_sync(0xffffffffu, key);
+  const int rank = __popc(same & ((1u << lane) - 1u));
+  __syncthreads();  // cnt is zero
+  if (live && rank == 0) cnt[warp][key] = __popc(same);
+  if (lane == 31) wsum[warp] = g_incl;
+  __syncthreads();
+  {
+    // key k = tid / 8: eight threads scan its counts over the warps, four warps each
+    const int k = tid >> 3, q = tid & 7;
+    int c[kWarps / 8];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < kWarps / 8; ++i) {
+      c[i] = cnt[(kWarps / 8) * q + i][k];
+      sum += c[i];
+    }
+    int sc = sum;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, sc, o, 8);
+      if (q >= o) sc += v;
+    }
+    int ex = sc - sum;
+#pragma unroll
+    for (int i = 0; i < kWarps / 8; ++i) {
+      cnt[(kWarps / 8) * q + i][k] = ex;
+      ex += c[i];
+    }
+    if (q == 7) total[k] = sc;
+  }
+  int g_total = 0;
+  if (warp == 0) {
+    // exclusive prefix of the warps' key_full units
+    const int w = wsum[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += v;
+    }
+    g_total = __shfl_sync(0xffffffffu, wi, 31);
+    __syncwarp();
+    wsum[lane] = wi - w;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // bucket starts, longest bucket first: lane l owns buckets 127-4l ... 124-4l
+    int c[kPlanBuckets / 32];
+    int mine = 0;
+#pragma unroll
+    for (int j = 0; j < kPlanBuckets / 32; ++j) {
+      const int k = kPlanBuckets - 1 - (kPlanBuckets / 32) * lane - j;
+      c[j] = k == key_full ? g_total : total[k];
+      mine += c[j];
+    }
+    int excl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, excl, o);
+      if (lane >= o) excl += v;
+    }
+    const int all = __shfl_sync(0xffffffffu, excl, 31);
+    excl -= mine;
+#pragma unroll
+    for (int j = 0; j < kPlanBuckets / 32; ++j) {
+      start[kPlanBuckets - 1 - (kPlanBuckets / 32) * lane - j] = excl;
+      excl += c[j];
+    }
+    if (lane == 0) {
+      counters[0] = 0;
+      counters[1] = all;
+    }
+  }
+  __syncthreads();
+  if (live) {
+    const int at_full = start[key_full] + wsum[warp] + g_incl - gv;
+    for (int p = 0; p < nfull; ++p) units[at_full + p] = make_uint2(((uint32_t)s << 16) | (uint32_t)p, ctx);
+    const int at = key == key_full ? at_full + nfull : start[key] + cnt[warp][key] + rank;
+    units[at] = make_uint2(((uint32_t)s << 16) | (uint32_t)(n - 1), ctx);
+  }
+}
+
 __global__ void __launch_bounds__(kPlanThreads)
     paged_decode_plan_kernel(const int32_t* __restrict__ context_lens, int num_seqs, int max_ctx, int part_tokens,
                              int sort, uint2* __restrict__ units, int* __restrict__ counters) {
   pdl_launch_dependents();
+  if (sort && num_seqs <= kPlanThreads) {
+    plan_sort_one_pass(context_lens, num_seqs, max_ctx, part_tokens, units, counters);
+    return;
+  }
   __shared__ int scratch[kPlanBuckets];
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;

@@ -58,6 +58,15 @@ constexpr int kKtPvWarp = 2 + kKtSoftmaxWarps;  // issues the P V products
 constexpr int kKtVWarp = 3 + kKtSoftmaxWarps;   // issues the V tiles' TMA loads
 constexpr int kKtThreads = (4 + kKtSoftmaxWarps) * 32;
 constexpr float kKtRescaleLog2 = 8.0f;
+// A softmax group's final output rows leave through one bulk copy per run of
+// consecutive rows (the rows of one query token are G consecutive query heads)
+// when that takes at most this many copies; otherwise, and for the strided rows
+// of partition states, the threads store them directly.  Measured on B200 (batch
+// 256, attention call): bulk copies ahead by 3-4 % with one or two runs (G = 8,
+// 32) and by ~1 % with two to four (G = 4 and 4 tokens, G = 2 and 8); direct
+// stores ahead by 2 % with eight runs (G = 1, 8 tokens), 7 % with sixteen (G = 1,
+// 32 tokens) and 11 % on 512-token partitions (G = 32).
+constexpr int kKtMaxBulkRuns = 4;
 
 // Instruction descriptor for kind::f16 with fp32 accumulation and either operand
 // MN-major (bit 15: A, bit 16: B).
@@ -374,15 +383,28 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
       return (long long)u < total_units ? __ldcg(prm.units + u / per_sp) : make_uint2(0u, 0u);
     };
 
+    // pool blocks of a tile's runs: lane l < units_per_tile reads the block of run l
+    auto run_blocks = [&](const TcUnit& d, int tile_t0) {
+      const int u_t0 = tile_t0 + lane * unit_rows;
+      return (lane < units_per_tile && u_t0 < d.t_end)
+                 ? __ldg(prm.block_tables + (size_t)d.s * prm.max_blocks + u_t0 / B)  // u_t0 < ctx <= max_blocks * B
+                 : -1;
+    };
+
     int u = (int)blockIdx.x;
     TcUnit cur = describe(u, entry(u));
+    // block-table entries are read one tile ahead (across unit boundaries too), so
+    // that their latency hides behind the previous tile's stage wait and loads
+    int phys_nx = run_blocks(cur, cur.t_begin);
     int it = 0;        // tiles issued
     // Query tiles (lane 0's bookkeeping): unit n's goes to buffer n % NQ once the S
-    // products of unit n - NQ are done.  A unit's tile is owed from the unit's
-    // start and issued as soon as its buffer is free, also while this warp waits
-    // for a stage, so the K/V tiles never wait for it.
+    // products of unit n - NQ are done.  A unit's tile is owed as soon as the unit
+    // is known (at the previous unit's last tile) and issued as soon as its buffer
+    // is free, also while this warp waits for a stage, so the K/V tiles never wait
+    // for it.  With one buffer (NQ = 1) only the first unit's is issued here; the
+    // S issuer issues each next one the moment the last S product frees the buffer.
     int nu = 0;        // query tiles issued
-    int owed = 0;      // units begun (query tiles owed up to this count)
+    int owed = 0;      // query tiles owed up to this count
     TcUnit q_unit = cur;
     auto q_ready = [&]() {
       return nu < NQ || mbar_test(&q_empty[nu % NQ], (uint32_t)(((nu / NQ) - 1) & 1));
@@ -406,42 +428,49 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
       q_issue();
       return true;
     };
+    // owe unit d's query tile (the previous one is issued first); false on a timeout
+    auto q_owe = [&](const TcUnit& d) {
+      int ok = 1;
+      if (lane == 0) {
+        ok = q_settle();
+        if (ok) {
+          q_unit = d;
+          ++owed;
+          if (q_ready()) q_issue();
+        }
+      }
+      return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    };
     bool stop = false;
+    if ((long long)u < total_units && !q_owe(cur)) stop = true;
     while (!stop) {
       const bool done = (long long)u >= total_units;
       const int u_next_lane0 = done ? 0 : claim();
       int u_next = 0;
       uint2 e_next = make_uint2(0u, 0u);
-      if (!done) {
-        // one query tile owed at a time: the previous unit's is issued first
-        int ok = 1;
-        if (lane == 0) {
-          ok = q_settle();
-          if (ok) {
-            q_unit = cur;
-            ++owed;
-            if (q_ready()) q_issue();
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-          if (lane == 0) {
-            flag_error(PKV_DEV_WAIT_TIMEOUT);
-            *abort_flag = 1;
-          }
-          break;
-        }
-      }
+      TcUnit nxt{0, 0, 0, 0, 0, 0, 1, 0};
       const int n_tok = max(0, cur.t_end - cur.t_begin);
       const int n_tiles = done ? 1 : max(1, (n_tok + kKtTile - 1) / kKtTile);
-      const int32_t* table = prm.block_tables + (size_t)cur.s * prm.max_blocks;
 
       for (int i = 0; i < n_tiles; ++i, ++it) {
         const int stage = it % NS;
         const int tile_t0 = cur.t_begin + i * kKtTile;
         const int u_t0 = tile_t0 + lane * unit_rows;
         const bool mine = !done && lane < units_per_tile && u_t0 < cur.t_end;
-        const int phys = mine ? __ldg(table + u_t0 / B) : -1;  // u_t0 < ctx <= max_blocks * B
+        const int phys = phys_nx;
+        // the next tile's blocks: this unit's next tile, or the next unit's first
+        // (its list entry was read at this unit's first tile; a one-tile unit reads
+        // them at the end of its tile)
+        bool next_known = false;
+        if (!done) {
+          if (i + 1 < n_tiles) {
+            phys_nx = run_blocks(cur, tile_t0 + kKtTile);
+          } else if (i > 0) {
+            nxt = describe(u_next, e_next);
+            phys_nx = run_blocks(nxt, nxt.t_begin);
+            next_known = true;
+          }
+        }
         if (it >= NS) {
           int ok = 1;
           if (lane == 0) {
@@ -462,10 +491,6 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) {
-            if (lane == 0) {
-              flag_error(PKV_DEV_WAIT_TIMEOUT);
-              *abort_flag = 1;
-            }
             stop = true;
             break;
           }
@@ -502,11 +527,24 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
         if (i == 0 && !done) {
           u_next = __shfl_sync(0xffffffffu, u_next_lane0, 0);
           e_next = entry(u_next);
+          if (n_tiles == 1) {
+            nxt = describe(u_next, e_next);
+            phys_nx = run_blocks(nxt, nxt.t_begin);
+            next_known = true;
+          }
+        }
+        if (NQ > 1 && next_known && (long long)u_next < total_units && !q_owe(nxt)) {
+          stop = true;
+          break;
         }
       }
       if (done || stop) break;
       u = u_next;
-      cur = describe(u, e_next);
+      cur = nxt;
+    }
+    if (stop && lane == 0) {
+      flag_error(PKV_DEV_WAIT_TIMEOUT);
+      *abort_flag = 1;
     }
     // the last unit's query tile, if still owed
     if (lane == 0 && !stop && !q_settle()) {
@@ -519,8 +557,10 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
       int no_abort = 0;
       for (int j = max(0, it - NS); j < it; ++j)
         if (!mbar_wait_bounded(&full[j % NS], (j / NS) & 1, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
-      for (int j = max(0, nu - NQ); j < nu; ++j)
-        if (!mbar_wait_bounded(&q_full[j % NQ], (j / NQ) & 1, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
+      // (with one query buffer the S issuer also loads it, and drains it)
+      if (NQ > 1)
+        for (int j = max(0, nu - NQ); j < nu; ++j)
+          if (!mbar_wait_bounded(&q_full[j % NQ], (j / NQ) & 1, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
     }
   } else if (warp == kKtVWarp) {
     // ------------------------------ V producer ------------------------------
@@ -558,7 +598,10 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
         constexpr uint32_t kIdescS = umma_idesc_ab<T>(kKtTile, NR, false, false);
         const uint64_t desc_k0 = umma_desc_sw128(smem_addr(smem), 16, 1024);
         const uint64_t desc_q0 = umma_desc_sw128(smem_addr(smem + Tr::kQOffset), 16, 1024);
+        const uint64_t policy = l2_evict_first();
         int nq = 0;  // query tiles consumed
+        // NQ = 1: query tiles issued (the producer issues the first unit's)
+        int nq_issued = (long long)blockIdx.x < total_units ? 1 : 0;
         for (int t = 0;; ++t) {
           const int stage = t % NS;
           if (!mbar_wait_bounded(&full[stage], (t / NS) & 1, abort_flag)) {
@@ -591,7 +634,34 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
             umma_f16(tmem_base + (uint32_t)(sb * NR), a0 + ka, b0 + kb, kIdescS, k > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[sb]);
-          if (flags & kTileLast) umma_commit(&q_empty[qb]);
+          if (flags & kTileLast) {
+            umma_commit(&q_empty[qb]);
+            if constexpr (NQ == 1) {
+              // The one query buffer is free once this product is done: load the
+              // next unit's rows (the next tile, published by the producer, opens it)
+              // right away rather than when the producer next looks.
+              const int tn = t + 1, sn = tn % NS;
+              if (!mbar_wait_bounded(&q_empty[0], (uint32_t)((nq - 1) & 1), abort_flag) ||
+                  !mbar_wait_bounded(&meta[sn], (uint32_t)((tn / NS) & 1), abort_flag)) {
+                ok = false;
+                break;
+              }
+              const int4 hn = hdr[2 * sn];
+              if (!((hn.w >> 16) & kTileEnd)) {
+                mbar_arrive_expect_tx(&q_full[0], (uint32_t)(2 * 128 * G * Tq));
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+                  tma_load_4d(smem + Tr::kQOffset + hf * Tr::kQSlab, &prm.tmap_q, hf * 64, (hn.y & 0xffff) * G,
+                              (hn.y >> 16) * Tq, hn.x, &q_full[0], policy);
+                ++nq_issued;
+              }
+            }
+          }
+        }
+        if (NQ == 1 && nq_issued > nq) {
+          // never leave with a query tile in flight into this CTA's shared memory
+          int no_abort = 0;
+          if (!mbar_wait_bounded(&q_full[0], (uint32_t)((nq_issued - 1) & 1), &no_abort)) ok = false;
         }
       } else {
         constexpr uint32_t kIdescO = umma_idesc_ab<T>(D, Tr::kPW, true, true);
@@ -888,10 +958,48 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
         const int us = hd.x, ukv = hd.y & 0xffff, up = hd.z & 0xffff, un = hd.z >> 16;
         const int rows = min(Tq, Lq - rt * Tq) * G;  // real rows of this tile
         const size_t row0 = (size_t)us * Lq + (size_t)rt * Tq;  // (sequence, first query token)
-        // The group's output rows go through the tile's V slabs (dead once P V is
-        // complete; the stage stays held until the rows are stored): thread tl
-        // writes dimension tl of each row, then one thread stores the rows with the
-        // copy engine, so no warp waits on scattered global stores.
+        if (un != 1 || NH > kKtMaxBulkRuns * G) {
+          // short runs: thread tl stores dimension tl of each row (a warp's store
+          // is 32 consecutive floats); the stage holds no output rows
+          if (warp == 2 + 4 * sg && lane == 0) mbar_arrive(&empty[stage]);
+          int tq = r0 / G, g = r0 - (r0 / G) * G;  // query token and head of row r0 + r
+#pragma unroll
+          for (int c = 0; c < NH / 8; ++c) {
+            uint32_t vh[8], vl[8];
+            tmem_ld8(tlane + Tr::kOCol + (uint32_t)(r0 + 8 * c), vh);
+            tmem_ld8(tlane + Tr::kOCol + (uint32_t)(Tr::kPW / 2 + r0 + 8 * c), vl);
+            tmem_wait_ld();
+            tmem_pin8(vh);
+            tmem_pin8(vl);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = 8 * c + i;
+              if (r0 + r < rows) {
+                const size_t sh = (row0 + tq) * prm.num_heads + (size_t)ukv * G + g;
+                const float v = __uint_as_float(vh[i]) + __uint_as_float(vl[i]);
+                if (un == 1)
+                  prm.out[sh * D + tl] = v * inv[r];
+                else
+                  prm.ws_acc[(sh * prm.max_parts + up) * D + tl] = v;
+              }
+              if (++g == G) {
+                g = 0;
+                ++tq;
+              }
+            }
+          }
+          if (un != 1 && tl < NH && r0 + tl < rows) {
+            const int R = r0 + tl;
+            const size_t sh = (row0 + R / G) * prm.num_heads + (size_t)ukv * G + R % G;
+            prm.ws_ml[sh * prm.max_parts + up] = make_float2(mref[tl], tmp[tl]);
+          }
+          tc_fence_before();
+          continue;
+        }
+        // Long runs (final rows): the group's rows go through the tile's V slabs
+        // (dead once P V is complete; the stage stays held until the rows are
+        // stored): thread tl writes dimension tl of each row, then one thread
+        // stores each run of rows with the copy engine.
         float* stg = reinterpret_cast<float*>(smem + stage * Tr::kStageBytes + 2 * Tr::kSlab) + sg * NH * D;
 #pragma unroll
         for (int c = 0; c < NH / 8; ++c) {
@@ -904,14 +1012,8 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int r = 8 * c + i;  // row r0 + r
-            const float v = __uint_as_float(vh[i]) + __uint_as_float(vl[i]);
-            stg[r * D + tl] = un == 1 ? v * inv[r] : v;
+            stg[r * D + tl] = (__uint_as_float(vh[i]) + __uint_as_float(vl[i])) * inv[r];
           }
-        }
-        if (un != 1 && tl < NH && r0 + tl < rows) {
-          const int R = r0 + tl;
-          const size_t sh = (row0 + R / G) * prm.num_heads + (size_t)ukv * G + R % G;
-          prm.ws_ml[sh * prm.max_parts + up] = make_float2(mref[tl], tmp[tl]);
         }
         fence_proxy_async_smem();  // the staged rows are read by the copy engine
         tc_fence_before();
@@ -920,21 +1022,14 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
           break;
         }
         if (warp == 2 + 4 * sg && lane == 0) {
+          // runs of rows of one query token are consecutive query heads
           const int r_end = min(r0 + NH, rows);
-          if (un == 1) {
-            // runs of rows of one query token are consecutive query heads
-            for (int R = r0; R < r_end;) {
-              const int tq = R / G, g = R - tq * G;
-              const int run = min(r_end - R, G - g);
-              bulk_store(prm.out + ((row0 + tq) * prm.num_heads + (size_t)ukv * G + g) * D, stg + (R - r0) * D,
-                         (uint32_t)(run * D * 4));
-              R += run;
-            }
-          } else {
-            for (int R = r0; R < r_end; ++R) {
-              const size_t sh = (row0 + R / G) * prm.num_heads + (size_t)ukv * G + R % G;
-              bulk_store(prm.ws_acc + (sh * prm.max_parts + up) * D, stg + (R - r0) * D, (uint32_t)(D * 4));
-            }
+          for (int R = r0; R < r_end;) {
+            const int tq = R / G, g = R - tq * G;
+            const int run = min(r_end - R, G - g);
+            bulk_store(prm.out + ((row0 + tq) * prm.num_heads + (size_t)ukv * G + g) * D, stg + (R - r0) * D,
+                       (uint32_t)(run * D * 4));
+            R += run;
           }
           bulk_commit();
           bulk_wait_read();

@@ -66,8 +66,10 @@ struct DecodePlan {
 // contexts of at most 512 tokens are never split.
 constexpr int kAutoPartitionTokens = 512;
 constexpr long long kRefCtas = 148 * 2;
-// Unit lists up to this length are ordered longest first by the plan kernel
-// (one warp, 32 sequences per step; the lengths are staged in shared memory).
+// The plan kernel orders the units longest first for up to kPlanThreads sequences
+// (one thread per sequence, any number of partitions) and for unit lists up to
+// this length (one warp, 32 sequences per step; the lengths are staged in shared
+// memory).
 constexpr long long kSortedUnitsMax = pkv::kPlanSortMaxSeqs;
 
 // H = partial-state rows per sequence (query heads x query tokens); Hkv = work
@@ -93,7 +95,7 @@ int make_plan(int S, int H, int Hkv, int D, int B, int MB, int requested, Decode
   plan->part_tokens = (int)pt;
   plan->max_parts = (int)parts;
   plan->split = parts > 1;
-  plan->sort = (long long)S * parts <= kSortedUnitsMax;
+  plan->sort = S <= pkv::kPlanThreads || (long long)S * parts <= kSortedUnitsMax;
   size_t off = 16;  // counters[2] (+ padding)
   plan->off_units = off;
   off += round16((size_t)S * parts * sizeof(uint2));

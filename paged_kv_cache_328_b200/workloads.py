@@ -203,9 +203,13 @@ def build_paged(context_lens, H, D, B, dtype, seed, *, device="cpu", num_blocks=
             pos = c - 1
             slot[s] = int(tables[s, pos // B]) * B + pos % B
             last[s] = starts[s] + pos
-    lastt = torch.from_numpy(last).to(device)
-    k_new = K_log.index_select(0, lastt)
-    v_new = V_log.index_select(0, lastt)
+    if total > 0:
+        lastt = torch.from_numpy(last).to(device)
+        k_new = K_log.index_select(0, lastt)
+        v_new = V_log.index_select(0, lastt)
+    else:  # no context holds a token: nothing to append (every slot is -1)
+        k_new = torch.zeros((S, H, D), dtype=K_log.dtype, device=device)
+        v_new = torch.zeros((S, H, D), dtype=V_log.dtype, device=device)
 
     return Workload(
         name=name, S=S, H=Hq, D=D, B=B, dtype=dtype, Hkv=H,

@@ -101,3 +101,13 @@ def test_last_block_waste():
     w = wl.make_tiny()
     blocks = 1 + 1 + 2 + 3
     assert math.isclose(wl.last_block_waste(w), 1 - (2 + 16 + 17 + 38) / (blocks * 16))
+
+
+def test_all_empty_contexts():
+    """A batch whose contexts are all empty has nothing to append: every slot is -1
+    and the append rows are zeros (no logical token exists to take them from)."""
+    for ctx in ([0], [0, 0, 0]):
+        w = wl.build_paged(np.array(ctx), 2, 64, 16, "f16", 3)
+        assert w.slot_mapping.tolist() == [-1] * len(ctx)
+        assert tuple(w.k_new.shape) == (len(ctx), 2, 64) and not bool(w.k_new.float().abs().sum())
+        assert bool(torch.isnan(w.k_pool.float()).all())
