@@ -178,37 +178,59 @@ __device__ __forceinline__ void rs_level(float* v, int lane, int off) {
 // share a row); the group's four warps meet in red[k & 1] ([row][warp]) after
 // phase k of the group's barrier.  Returns false if that wait failed (abort or
 // timeout).
+// Reduce-scatter of 32 values over the warp: lane l returns the warp's partial of value l.
+template <bool kMax>
+__device__ __forceinline__ float warp_rs32(const float* v, int lane) {
+  float w[16];
+  const bool up = (lane & 16) != 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float send = up ? v[i] : v[i + 16];
+    const float keep = up ? v[i + 16] : v[i];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+    w[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+  rs_level<16, kMax>(w, lane, 8);
+  rs_level<8, kMax>(w, lane, 4);
+  rs_level<4, kMax>(w, lane, 2);
+  rs_level<2, kMax>(w, lane, 1);
+  return w[0];
+}
+
 template <int N, bool kMax>
 __device__ __forceinline__ bool group_reduce(const float (&v)[N], float* red, float* out, uint64_t* grp, int& k,
                                              int q4, int lane, volatile int* abort_flag) {
   static_assert(N == 8 || N == 16 || N == 32, "8, 16 or 32 rows per group");
-  float w[N / 2];
-  {
-    const bool up = (lane & 16) != 0;
-#pragma unroll
-    for (int i = 0; i < N / 2; ++i) {
-      const float send = up ? v[i] : v[i + N / 2];
-      const float keep = up ? v[i + N / 2] : v[i];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-      w[i] = kMax ? fmaxf(keep, recv) : keep + recv;
-    }
-  }
-  if constexpr (N >= 4) rs_level<N / 2, kMax>(w, lane, 8);
-  if constexpr (N >= 8) rs_level<N / 4, kMax>(w, lane, 4);
-  if constexpr (N >= 16) rs_level<N / 8, kMax>(w, lane, 2);
-  if constexpr (N >= 32) rs_level<N / 16, kMax>(w, lane, 1);
-  // lanes that hold the same row (N < 32) finish with a butterfly all-reduce
-  if constexpr (N <= 16) {
-    const float o = __shfl_xor_sync(0xffffffffu, w[0], 1);
-    w[0] = kMax ? fmaxf(w[0], o) : w[0] + o;
-  }
-  if constexpr (N <= 8) {
-    const float o = __shfl_xor_sync(0xffffffffu, w[0], 2);
-    w[0] = kMax ? fmaxf(w[0], o) : w[0] + o;
-  }
   float* buf = red + (k & 1) * N * 4;
-  constexpr int kShare = 32 / N;  // lanes per row (N <= 32)
-  if (lane % kShare == 0) buf[(lane / kShare) * 4 + q4] = w[0];
+  if constexpr (N == 32) {
+    buf[lane * 4 + q4] = warp_rs32<kMax>(v, lane);  // lane l holds row l
+  } else {
+    float w[N / 2];
+    {
+      const bool up = (lane & 16) != 0;
+#pragma unroll
+      for (int i = 0; i < N / 2; ++i) {
+        const float send = up ? v[i] : v[i + N / 2];
+        const float keep = up ? v[i + N / 2] : v[i];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+        w[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+      }
+    }
+    rs_level<N / 2, kMax>(w, lane, 8);
+    if constexpr (N >= 8) rs_level<N / 4, kMax>(w, lane, 4);
+    if constexpr (N >= 16) rs_level<N / 8, kMax>(w, lane, 2);
+    // lanes that hold the same row (N < 32) finish with a butterfly all-reduce
+    {
+      const float o = __shfl_xor_sync(0xffffffffu, w[0], 1);
+      w[0] = kMax ? fmaxf(w[0], o) : w[0] + o;
+    }
+    if constexpr (N <= 8) {
+      const float o = __shfl_xor_sync(0xffffffffu, w[0], 2);
+      w[0] = kMax ? fmaxf(w[0], o) : w[0] + o;
+    }
+    constexpr int kShare = 32 / N;  // lanes per row
+    if (lane % kShare == 0) buf[(lane / kShare) * 4 + q4] = w[0];
+  }
   __syncwarp();
   if (lane == 0) mbar_arrive(grp);
   const bool ok = __all_sync(0xffffffffu, mbar_spin_bounded(grp, (uint32_t)(k & 1), abort_flag));
@@ -783,12 +805,21 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
       // every row of the group sees every token of the warp: no masking needed
       const bool open = __all_sync(0xffffffffu, r_lo <= r0 && r_hi >= r0 + NH);
 
+      // rows this thread's token is hidden from get t = -inf (after the scaling,
+      // so that a row no token sees, whose m_r is -inf, cannot turn into +inf)
+      auto mask_hidden = [&]() {
+        if (!open) {
+          const int lo = r_lo - r0, hi = r_hi - r0;  // visible rows of this group: [lo, hi)
+#pragma unroll
+          for (int r = 0; r < NH; ++r) x[r] = (r >= lo && r < hi) ? x[r] : -INFINITY;
+        }
+      };
       // t = x * scale - m_r (log2 units, -inf where masked)
       if (flags & kTileFirst) {
         // the unit's reference maxima: this tile's row maxima
 #pragma unroll
-        for (int r = 0; r < NH; ++r)
-          x[r] = (open || (r0 + r >= r_lo && r0 + r < r_hi)) ? x[r] * scale : -INFINITY;
+        for (int r = 0; r < NH; ++r) x[r] *= scale;
+        mask_hidden();
         if (!group_reduce<NH, true>(x, red, mref, my_grp, gk, q4, lane, abort_flag)) {
           failed = true;
           break;
@@ -805,31 +836,19 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
           }
         }
       } else {
-        float tmax = -INFINITY;
-        if (open) {
+        // a row that some token sees has a finite m_r (visibility is a prefix of the partition)
 #pragma unroll
-          for (int c = 0; c < NH / 4; ++c) {
-            const float4 m = mref4[c];
-            x[4 * c] = fmaf(x[4 * c], scale, -m.x);
-            x[4 * c + 1] = fmaf(x[4 * c + 1], scale, -m.y);
-            x[4 * c + 2] = fmaf(x[4 * c + 2], scale, -m.z);
-            x[4 * c + 3] = fmaf(x[4 * c + 3], scale, -m.w);
-            tmax = fmaxf(tmax, fmaxf(fmaxf(x[4 * c], x[4 * c + 1]), fmaxf(x[4 * c + 2], x[4 * c + 3])));
-          }
-        } else {
-          // a row that some token sees has a finite m_r (visibility is a prefix of the partition)
-#pragma unroll
-          for (int c = 0; c < NH / 4; ++c) {
-            const float4 m = mref4[c];
-            const float mm[4] = {m.x, m.y, m.z, m.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int r = 4 * c + i;
-              x[r] = (r0 + r >= r_lo && r0 + r < r_hi) ? fmaf(x[r], scale, -mm[i]) : -INFINITY;
-              tmax = fmaxf(tmax, x[r]);
-            }
-          }
+        for (int c = 0; c < NH / 4; ++c) {
+          const float4 m = mref4[c];
+          x[4 * c] = fmaf(x[4 * c], scale, -m.x);
+          x[4 * c + 1] = fmaf(x[4 * c + 1], scale, -m.y);
+          x[4 * c + 2] = fmaf(x[4 * c + 2], scale, -m.z);
+          x[4 * c + 3] = fmaf(x[4 * c + 3], scale, -m.w);
         }
+        mask_hidden();
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < NH; ++r) tmax = fmaxf(tmax, x[r]);
         bool ok = true;
         const bool need = group_any(tmax > kKtRescaleLog2, vote, my_grp, gk, q4, lane, abort_flag, ok);
         if (!ok) {
@@ -849,7 +868,6 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
             mref[lane] += d;
           }
           __syncwarp();
-          float alpha[NH];
 #pragma unroll
           for (int c = 0; c < NH / 4; ++c) {
             const float4 dd = tmp4[c];
@@ -858,8 +876,7 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
             for (int i = 0; i < 4; ++i) {
               const int r = 4 * c + i;
               x[r] -= dv[i];
-              alpha[r] = ex2_fast(-dv[i]);
-              lpart[r] *= alpha[r];
+              lpart[r] *= ex2_fast(-dv[i]);
             }
           }
           // O holds every product of this unit issued so far: all must be complete
@@ -878,7 +895,7 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
               tmem_wait_ld();
               tmem_pin8(v);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha[8 * c + i]);
+              for (int i = 0; i < 8; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * ex2_fast(-tmp[8 * c + i]));
               tmem_st8(col, v);
             }
           }
