@@ -15,6 +15,9 @@ __global__ void __launch_bounds__(kAppendThreads)
     kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, uint4* __restrict__ k_cache,
                      uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int num_heads,
                      int row_vecs, int block_size, long long num_slots) {
+  // a programmatic dependent (the decode plan) may start now: it reads nothing
+  // this kernel writes, and waits for it to complete before its own writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int t = blockIdx.x;
   const int is_v = blockIdx.y;
   const long long slot = slot_mapping[t];

@@ -122,7 +122,11 @@ __device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontro
 //    adjacent and their shared blocks are re-read from L2.  Longest-first lets
 //    the dynamically scheduled CTAs end together.  Up to kPlanThreads sequences
 //    are placed in one pass, one thread per sequence; longer lists take one warp
-//    over runs of 32 sequences.
+//    over runs of 32 sequences.  The plan is a programmatic dependent launch: it
+//    reads the lengths and sorts while the stream's previous kernel finishes (our
+//    kernels let dependents start early; none writes the lengths), and waits for
+//    that kernel before its first write, so it never changes the list or the
+//    counters under a previous call's decode kernel.
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 128;
@@ -225,6 +229,8 @@ __device__ __forceinline__ void plan_sort_one_pass(const int32_t* __restrict__ c
     wsum[lane] = wi - w;
   }
   __syncthreads();
+  // the previous call's kernels may still read the list and the counters
+  pdl_wait_primary();
   if (warp == 0) {
     // bucket starts, longest bucket first: lane l owns buckets 127-4l ... 124-4l
     int c[kPlanBuckets / 32];
@@ -285,6 +291,7 @@ __global__ void __launch_bounds__(kPlanThreads)
     for (int k = tid; k < kPlanBuckets; k += kPlanThreads) scratch[k] = 0;
     __syncthreads();
     if (warp != 0) return;
+    pdl_wait_primary();  // the previous call's kernels may still read the list and the counters
     const unsigned below = (1u << lane) - 1u;
     const int key_full = unit_bucket(part_tokens);  // every partition but a sequence's last is full
     // pass 0 counts the units of each bucket; pass 1 places them.  A run of 32
@@ -371,6 +378,7 @@ __global__ void __launch_bounds__(kPlanThreads)
   }
   if (lane == 31) scratch[warp] = incl;
   __syncthreads();
+  pdl_wait_primary();  // the previous call's kernels may still read the list and the counters
   if (warp == 0) {
     const int w = scratch[lane];
     int wi = w;

@@ -535,6 +535,27 @@ int launch_kt_path(const void* q, const void* k_cache, const void* v_cache, cons
   return bf ? launch_kt<__nv_bfloat16, 64>(t, max_units, st) : launch_kt<__half, 64>(t, max_units, st);
 }
 
+// The plan kernel is a programmatic dependent of the stream's previous kernel: it
+// reads the context lengths and sorts while that kernel finishes, and waits for it
+// before writing the unit list and the counters.
+int launch_plan(const int32_t* context_lens, int num_seqs, int max_ctx, const DecodePlan& plan, uint2* units,
+                int* counters, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(pkv::kPlanThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, pkv::paged_decode_plan_kernel, context_lens, num_seqs, max_ctx, plan.part_tokens,
+                         plan.sort ? 1 : 0, units, counters) != cudaSuccess)
+    return PKV_ECUDA;
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
 // The merge is a programmatic dependent of the decode kernel: its CTAs may be
 // scheduled as decode CTAs run out of units and wait for the decode to finish.
 template <int D>
@@ -665,10 +686,9 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const i
 
   const int max_ctx = max_blocks_per_seq * block_size;
   int result = PKV_OK;
-  pkv::paged_decode_plan_kernel<<<1, pkv::kPlanThreads, 0, st>>>(
-      context_lens, num_seqs, max_ctx, plan.part_tokens, plan.sort ? 1 : 0,
-      reinterpret_cast<uint2*>(ws + plan.off_units), prm.counters);
-  if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
+  if (launch_plan(context_lens, num_seqs, max_ctx, plan, reinterpret_cast<uint2*>(ws + plan.off_units), prm.counters,
+                  st) != PKV_OK)
+    result = PKV_ECUDA;
   const int group = num_heads / num_kv_heads;
   const bool tc_ok = dtype != PKV_F32 && group >= 2 && (long long)num_blocks * num_kv_heads * block_size < (1LL << 31);
   if (result == PKV_OK && tc_ok && tc_path(1, group, head_dim) == TcPath::kKt) {
@@ -743,10 +763,9 @@ int multi_query_impl(const void* q, const void* k_cache, const void* v_cache, co
   prm.counters = reinterpret_cast<int*>(ws);
   const int max_ctx = max_blocks_per_seq * block_size;
   int result = PKV_OK;
-  pkv::paged_decode_plan_kernel<<<1, pkv::kPlanThreads, 0, st>>>(
-      context_lens, num_seqs, max_ctx, plan.part_tokens, plan.sort ? 1 : 0,
-      reinterpret_cast<uint2*>(ws + plan.off_units), prm.counters);
-  if (cudaGetLastError() != cudaSuccess) result = PKV_ECUDA;
+  if (launch_plan(context_lens, num_seqs, max_ctx, plan, reinterpret_cast<uint2*>(ws + plan.off_units), prm.counters,
+                  st) != PKV_OK)
+    result = PKV_ECUDA;
   const TcPath path = tc_path(q_len, num_heads / num_kv_heads, head_dim);
   if (result == PKV_OK && path == TcPath::kKt)
     result = launch_kt_path(q, k_cache, v_cache, block_tables, num_seqs, q_len, num_heads, num_kv_heads, head_dim,
