@@ -28,8 +28,10 @@
 // Warp roles (one CTA per SM, persistent over the unit list):
 //   warp 0     producer: the unit's query tile (one 4-D TMA box per 64 columns) and
 //              the K/V tiles (2-D TMA boxes per (block, K/V head) run, 128-byte swizzle);
-//   warp 1     allocates / frees the tensor memory; its lane 0 issues every MMA and
-//              commits completion to mbarriers;
+//   warp 1     allocates / frees the tensor memory; its lane 0 issues the S products;
+//   warp 6     its lane 0 issues the P V products, in tile order, as each P is written
+//              (the two issuers commit to their own barriers, so neither waits behind
+//              the other's issue);
 //   warps 2-5  softmax and epilogue; warp w reads tensor-memory lanes 32*(w%4) ...
 //
 // Every mbarrier wait is bounded (kWaitLimitCycles) and checks the CTA abort flag;
@@ -43,7 +45,8 @@ namespace pkv {
 constexpr int kTcRows = 128;          // M: query rows per tile = tensor-memory lanes
 constexpr int kTcTile = 64;           // tokens per K/V tile
 constexpr int kTcStages = 6;  // the P V product of tile t is issued after S of tile t + 2
-constexpr int kTcThreads = 6 * 32;    // producer, MMA, four softmax warps
+constexpr int kTcThreads = 7 * 32;    // producer, S issuer, four softmax warps, P V issuer
+constexpr int kTcPvWarp = 6;
 constexpr int kTcCtasPerSm = 1;       // shared memory (and tensor memory) per CTA
 constexpr int kTcTmemCols = 512;      // S[2] at columns 0 and 64, O at 128, P[2] (high, low) at 256 and 320
 constexpr float kTcRescaleLog2 = 8.0f;
@@ -82,8 +85,8 @@ struct TcTraits {
   static constexpr int kQOffset = kTcStages * kStageBytes;
   static constexpr int kHdrOffset = kQOffset + kHalves * kQSlabBytes;  // two int4 per stage
   static constexpr int kBarOffset = kHdrOffset + kTcStages * 32;
-  // full[NS], empty[NS], q_full, q_empty, s_full[2], s_free[2], p_full[2], o_done[2], drain
-  static constexpr int kNumBars = 2 * kTcStages + 11;
+  // full[NS], empty[NS], q_full, q_empty, s_full[2], s_free[2], p_full[2], o_done[2], drain[2]
+  static constexpr int kNumBars = 2 * kTcStages + 12;
   static constexpr int kTmemSlotOffset = kBarOffset + kNumBars * 8;
   static constexpr int kAbortOffset = kTmemSlotOffset + 8;
   static constexpr int kSmemBytes = kAbortOffset + 8;
@@ -258,7 +261,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
   uint64_t* s_free = q_full + 4;  // [2]
   uint64_t* p_full = q_full + 6;  // [2]: P buffer b of tile j = j & 1 written
   uint64_t* o_done = q_full + 8;  // [2]: P V of tile j (j & 1 = b) complete
-  uint64_t* drain = q_full + 10;
+  uint64_t* drain = q_full + 10;  // [2]: one per MMA issuer
   int4* hdr = reinterpret_cast<int4*>(smem + Tr::kHdrOffset);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::kTmemSlotOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Tr::kAbortOffset);
@@ -287,7 +290,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
     mbar_init(&p_full[1], 4);
     mbar_init(&o_done[0], 1);
     mbar_init(&o_done[1], 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -437,96 +441,89 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
           flag_error(PKV_DEV_WAIT_TIMEOUT);
       if (nu > 0 && !mbar_wait_bounded(q_full, (nu - 1) & 1, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
     }
-  } else if (warp == 1) {
-    // ----------------------------- MMA issuer -----------------------------
+  } else if (warp == 1 || warp == kTcPvWarp) {
+    // ----------------------------- MMA issuers -----------------------------
     if (lane == 0) {
       constexpr uint32_t kIdescS = umma_idesc<T>(kTcRows, kTcTile, false);
       constexpr uint32_t kIdescO = umma_idesc<T>(kTcRows, D, true);
       const uint32_t q_base = smem_addr(smem + Tr::kQOffset);
-
       bool ok = true;
-      int nu = 0;
-      // O += P V for the tile issued one step earlier
-      auto pv = [&](int it_prev, int stage_prev, bool first_prev) {
-        const int pb = it_prev & 1;
-        if (!mbar_wait_bounded(&p_full[pb], (it_prev >> 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t p_hi = tmem_base + Tr::kPCol + (uint32_t)(pb * 64);
-        const uint32_t p_lo = p_hi + 32;
-        const uint32_t v_base = smem_addr(smem + stage_prev * Tr::kStageBytes + Tr::kTileBytes);
-#pragma unroll
-        for (int k = 0; k < kTcTile / 16; ++k) {  // 16 tokens = 8 columns of packed pairs
-          const uint64_t b = umma_desc_sw128(v_base + k * 16 * 128, Tr::kSlabBytes, 1024);
-          umma_f16_tmem_a(tmem_base + Tr::kOCol, p_hi + 8 * k, b, kIdescO, (first_prev && k == 0) ? 0u : 1u);
-          umma_f16_tmem_a(tmem_base + Tr::kOCol, p_lo + 8 * k, b, kIdescO, 1u);
-        }
-        umma_commit(&empty[stage_prev]);
-        umma_commit(&o_done[pb]);
-        return true;
-      };
-      // S of tile t is issued as soon as its K/V and S buffer are ready; the P V
-      // product of tile t - 2 follows it (of tile t - 1 too when tile t opens a new
-      // unit, whose epilogue reads O), so the tensor pipe always holds an S product
-      // ahead of the softmax warps.
-      int it = 0;
-      int pv_next = 0;               // first tile whose P V product is not issued
-      bool first_of[2] = {false, false};  // first-tile flags of the tiles in flight, by t & 1
-      auto pv_upto = [&](int t_last) {
-        while (ok && pv_next <= t_last) {
-          const bool f = (pv_next & 1) ? first_of[1] : first_of[0];
-          if (!pv(pv_next, pv_next % kTcStages, f)) ok = false;
-          ++pv_next;
-        }
-      };
-      while (ok) {
-        const int stage = it % kTcStages;
-        if (!mbar_wait_bounded(&full[stage], (it / kTcStages) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const int flags = hdr[2 * stage].w >> 16;
-        if (flags & kTileEnd) break;
-        const bool first = flags & kTileFirst;
-        if (first) {
-          if (!mbar_wait_bounded(q_full, nu & 1, abort_flag)) {
+      if (warp == 1) {
+        // S of tile t as soon as its K/V, the unit's query tile and its S buffer are ready
+        int nu = 0;
+        for (int it = 0;; ++it) {
+          const int stage = it % kTcStages;
+          if (!mbar_wait_bounded(&full[stage], (it / kTcStages) & 1, abort_flag)) {
             ok = false;
             break;
           }
-          ++nu;
-        }
-        const int sb = it & 1;
-        if (it >= 2 && !mbar_wait_bounded(&s_free[sb], ((it >> 1) - 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t k_base = smem_addr(smem + stage * Tr::kStageBytes);
+          const int flags = hdr[2 * stage].w >> 16;
+          if (flags & kTileEnd) break;
+          if (flags & kTileFirst) {
+            if (!mbar_wait_bounded(q_full, nu & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            ++nu;
+          }
+          const int sb = it & 1;
+          if (it >= 2 && !mbar_wait_bounded(&s_free[sb], ((it >> 1) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t k_base = smem_addr(smem + stage * Tr::kStageBytes);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (uint32_t)(k & 3) * 32u;  // 16 columns = 32 bytes inside a slab
-          const uint64_t a = umma_desc_sw128(q_base + (k >> 2) * Tr::kQSlabBytes + off, 16, 1024);
-          const uint64_t b = umma_desc_sw128(k_base + (k >> 2) * Tr::kSlabBytes + off, 16, 1024);
-          umma_f16(tmem_base + (uint32_t)(sb * kTcTile), a, b, kIdescS, k > 0 ? 1u : 0u);
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (uint32_t)(k & 3) * 32u;  // 16 columns = 32 bytes inside a slab
+            const uint64_t a = umma_desc_sw128(q_base + (k >> 2) * Tr::kQSlabBytes + off, 16, 1024);
+            const uint64_t b = umma_desc_sw128(k_base + (k >> 2) * Tr::kSlabBytes + off, 16, 1024);
+            umma_f16(tmem_base + (uint32_t)(sb * kTcTile), a, b, kIdescS, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[sb]);
+          if (flags & kTileLast) umma_commit(q_empty);
         }
-        umma_commit(&s_full[sb]);
-        if (flags & kTileLast) umma_commit(q_empty);
-        // tiles t - 2 and t share a history slot: issue the pending products first
-        pv_upto(first ? it - 1 : it - 2);
-        if (sb)
-          first_of[1] = first;
-        else
-          first_of[0] = first;
-        ++it;
+      } else {
+        // O += P V of tile t once its P is written; a unit's first tile starts O over
+        // (the softmax writes that P only after the previous unit's rows are read)
+        for (int it = 0;; ++it) {
+          const int stage = it % kTcStages;
+          // the stage is released by this thread's commit below, so its header stays valid
+          if (!mbar_wait_bounded(&full[stage], (it / kTcStages) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int flags = hdr[2 * stage].w >> 16;
+          if (flags & kTileEnd) break;
+          const int pb = it & 1;
+          if (!mbar_wait_bounded(&p_full[pb], (it >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const bool first = flags & kTileFirst;
+          const uint32_t p_hi = tmem_base + Tr::kPCol + (uint32_t)(pb * 64);
+          const uint32_t p_lo = p_hi + 32;
+          const uint32_t v_base = smem_addr(smem + stage * Tr::kStageBytes + Tr::kTileBytes);
+#pragma unroll
+          for (int k = 0; k < kTcTile / 16; ++k) {  // 16 tokens = 8 columns of packed pairs
+            const uint64_t b = umma_desc_sw128(v_base + k * 16 * 128, Tr::kSlabBytes, 1024);
+            umma_f16_tmem_a(tmem_base + Tr::kOCol, p_hi + 8 * k, b, kIdescO, (first && k == 0) ? 0u : 1u);
+            umma_f16_tmem_a(tmem_base + Tr::kOCol, p_lo + 8 * k, b, kIdescO, 1u);
+          }
+          umma_commit(&empty[stage]);
+          umma_commit(&o_done[pb]);
+        }
       }
-      if (ok) pv_upto(it - 1);
       if (!ok) {
         flag_error(PKV_DEV_WAIT_TIMEOUT);
         *abort_flag = 1;
       }
-      // every MMA issued above must be complete before the tensor memory is freed
-      umma_commit(drain);
+      // every MMA this thread issued must be complete before the tensor memory is freed
+      uint64_t* my_drain = warp == 1 ? &drain[0] : &drain[1];
+      umma_commit(my_drain);
       int no_abort = 0;
-      if (!mbar_wait_bounded(drain, 0, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
+      if (!mbar_wait_bounded(my_drain, 0, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
     }
     __syncwarp();
   } else {
