@@ -27,7 +27,9 @@
 //
 // Warp roles (one CTA per SM, persistent over the unit list):
 //   warp 0     producer: the unit's query tile (one 4-D TMA box per 64 columns) and
-//              the K/V tiles (2-D TMA boxes per (block, K/V head) run, 128-byte swizzle);
+//              the K half of each tile (2-D TMA boxes per (block, K/V head) run,
+//              128-byte swizzle); it publishes each tile's header and run rows;
+//   warp 7     V producer: the V half of each published tile, on the same barrier;
 //   warp 1     allocates / frees the tensor memory; its lane 0 issues the S products;
 //   warp 6     its lane 0 issues the P V products, in tile order, as each P is written
 //              (the two issuers commit to their own barriers, so neither waits behind
@@ -45,8 +47,9 @@ namespace pkv {
 constexpr int kTcRows = 128;          // M: query rows per tile = tensor-memory lanes
 constexpr int kTcTile = 64;           // tokens per K/V tile
 constexpr int kTcStages = 6;  // the P V product of tile t is issued after S of tile t + 2
-constexpr int kTcThreads = 7 * 32;    // producer, S issuer, four softmax warps, P V issuer
+constexpr int kTcThreads = 8 * 32;    // producer, S issuer, four softmax warps, P V issuer, V producer
 constexpr int kTcPvWarp = 6;
+constexpr int kTcVWarp = 7;
 constexpr int kTcCtasPerSm = 1;       // shared memory (and tensor memory) per CTA
 constexpr int kTcTmemCols = 512;      // S[2] at columns 0 and 64, O at 128, P[2] (high, low) at 256 and 320
 constexpr float kTcRescaleLog2 = 8.0f;
@@ -84,9 +87,10 @@ struct TcTraits {
   static constexpr int kQSlabBytes = kTcRows * 128;         // 128 rows x 64 columns
   static constexpr int kQOffset = kTcStages * kStageBytes;
   static constexpr int kHdrOffset = kQOffset + kHalves * kQSlabBytes;  // two int4 per stage
-  static constexpr int kBarOffset = kHdrOffset + kTcStages * 32;
-  // full[NS], empty[NS], q_full, q_empty, s_full[2], s_free[2], p_full[2], o_done[2], drain[2]
-  static constexpr int kNumBars = 2 * kTcStages + 12;
+  static constexpr int kRowsOffset = kHdrOffset + kTcStages * 32;  // [NS][32] pool rows of a tile's runs (-1: none)
+  static constexpr int kBarOffset = kRowsOffset + kTcStages * 128;
+  // full[NS], empty[NS], q_full, q_empty, s_full[2], s_free[2], p_full[2], o_done[2], drain[2], meta[NS]
+  static constexpr int kNumBars = 3 * kTcStages + 12;
   static constexpr int kTmemSlotOffset = kBarOffset + kNumBars * 8;
   static constexpr int kAbortOffset = kTmemSlotOffset + 8;
   static constexpr int kSmemBytes = kAbortOffset + 8;
@@ -262,6 +266,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
   uint64_t* p_full = q_full + 6;  // [2]: P buffer b of tile j = j & 1 written
   uint64_t* o_done = q_full + 8;  // [2]: P V of tile j (j & 1 = b) complete
   uint64_t* drain = q_full + 10;  // [2]: one per MMA issuer
+  uint64_t* meta = q_full + 12;   // [NS]: a tile's header and run rows are published
+  int* run_rows = reinterpret_cast<int*>(smem + Tr::kRowsOffset);
   int4* hdr = reinterpret_cast<int4*>(smem + Tr::kHdrOffset);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::kTmemSlotOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Tr::kAbortOffset);
@@ -279,6 +285,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
     for (int i = 0; i < kTcStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
+      mbar_init(&meta[i], 1);
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
@@ -406,22 +413,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
             flag_error(PKV_DEV_BLOCK_ID);
         }
         const unsigned loads = __ballot_sync(0xffffffffu, load);
+        const int y = load ? (phys * Hkv + cur.kvh) * B + (u_t0 % B) : -1;
+        // publish the tile (header, pool row of each run) for the V producer, arm the
+        // stage's barrier with the bytes of both halves, then load the K half
+        run_rows[stage * 32 + lane] = y;
         if (lane == 0) {
           const int flags = done ? kTileEnd : ((i == 0 ? kTileFirst : 0) | (i == n_tiles - 1 ? kTileLast : 0));
           hdr[2 * stage] = make_int4(cur.s, cur.kvh | (cur.rt << 16), cur.p | (cur.n_parts << 16),
                                      n_valid | (flags << 16));
           hdr[2 * stage + 1] = make_int4(tile_t0, cur.ctx, 0, 0);
-          mbar_arrive_expect_tx(&full[stage], (uint32_t)__popc(loads) * 2u * Tr::kHalves * run_bytes);
         }
         __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[stage], (uint32_t)__popc(loads) * 2u * Tr::kHalves * run_bytes);
+          mbar_arrive(&meta[stage]);
+        }
         if (load) {
-          const int y = (phys * Hkv + cur.kvh) * B + (u_t0 % B);
           unsigned char* kt = smem + stage * Tr::kStageBytes + lane * unit_rows * 128;
 #pragma unroll
-          for (int hf = 0; hf < Tr::kHalves; ++hf) {
+          for (int hf = 0; hf < Tr::kHalves; ++hf)
             tma_load_2d(kt + hf * Tr::kSlabBytes, &prm.tmap_k, hf * 64, y, &full[stage], policy);
-            tma_load_2d(kt + Tr::kTileBytes + hf * Tr::kSlabBytes, &prm.tmap_v, hf * 64, y, &full[stage], policy);
-          }
         }
         if (i == 0 && !done) {
           u_next = __shfl_sync(0xffffffffu, u_next_lane0, 0);
@@ -440,6 +451,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
         if (!mbar_wait_bounded(&full[j % kTcStages], (j / kTcStages) & 1, &no_abort))
           flag_error(PKV_DEV_WAIT_TIMEOUT);
       if (nu > 0 && !mbar_wait_bounded(q_full, (nu - 1) & 1, &no_abort)) flag_error(PKV_DEV_WAIT_TIMEOUT);
+    }
+  } else if (warp == kTcVWarp) {
+    // ------------------------------ V producer ------------------------------
+    // Follows the producer tile by tile: once a tile is published (meta), each run's V
+    // rows go to the stage's V half, completing on the same barrier.
+    const uint64_t policy = l2_evict_first();
+    const int unit_rows = min(prm.block_size, kTcTile);
+    for (int t = 0;; ++t) {
+      const int stage = t % kTcStages;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&meta[stage], (t / kTcStages) & 1, abort_flag))) {
+        if (lane == 0) {
+          flag_error(PKV_DEV_WAIT_TIMEOUT);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      if ((hdr[2 * stage].w >> 16) & kTileEnd) break;
+      const int y = run_rows[stage * 32 + lane];
+      if (y >= 0) {
+        unsigned char* vt = smem + stage * Tr::kStageBytes + Tr::kTileBytes + lane * unit_rows * 128;
+#pragma unroll
+        for (int hf = 0; hf < Tr::kHalves; ++hf)
+          tma_load_2d(vt + hf * Tr::kSlabBytes, &prm.tmap_v, hf * 64, y, &full[stage], policy);
+      }
     }
   } else if (warp == 1 || warp == kTcPvWarp) {
     // ----------------------------- MMA issuers -----------------------------
