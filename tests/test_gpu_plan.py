@@ -119,3 +119,38 @@ def test_long_lists(dev, S, pt, sorted_list):
                               w.scale, B, "f16")
     assert np.all(np.isfinite(got))
     assert max_err(got, ref) <= TOL["f16"]
+
+
+@pytest.mark.parametrize("H,Hq", [(8, 8), (2, 64), (2, 16)])
+def test_back_to_back_calls_share_one_workspace(dev, H, Hq):
+    """Calls queued back to back on one stream and one workspace, with different context
+    lengths and partition sizes: each call's plan reads its lengths while the previous
+    call's kernels may still run and must not change the unit list or the counters under
+    them (the plan waits for its predecessor before writing).  MHA, the token-major and the
+    warp-level grouped-query kernels; every output against the oracle."""
+    B, mb, S = 16, 64, 96
+    rng = np.random.default_rng(1200 + Hq)
+    ctx_sets = [rng.integers(0, mb * B + 1, S) for _ in range(3)]
+    ctx_sets[1][:5] = 0
+    w = wl.build_paged(ctx_sets[0], H=H, D=128, B=B, dtype="bf16", seed=1201 + Hq, device=dev, max_blocks=mb,
+                       num_q_heads=Hq)
+    ix = dev_indices(w, dev)
+    ws = pkv.alloc_workspace(w.q, w.k_pool, ix["bt"], 64)  # the largest of the plans below
+    calls = [(ctx_sets[i % 3], pt) for i, pt in enumerate([0, 64, 256, 0, 512, 64, 0, 256, 1024])]
+    # inputs and outputs made first, so nothing but the calls themselves sits between them
+    ctx_dev = [torch.from_numpy(c.astype(np.int32)).to(dev) for c in ctx_sets]
+    outs = [torch.full((w.S, w.H, w.D), float("nan"), dtype=torch.float32, device=dev) for _ in calls]
+    ws.fill_(0xFF)
+    torch.cuda.synchronize()
+    for k, (_, pt) in enumerate(calls):
+        pkv.paged_attn_decode(w.q, w.k_pool, w.v_pool, ix["bt"], ctx_dev[k % 3], w.scale, out=outs[k],
+                              partition_tokens=pt, workspace=ws)
+    torch.cuda.synchronize()
+    code, reason = pkv.get_device_error(dev)
+    assert code == 0, (code, reason)
+    want = {i: oracle.paged_decode(w.host(w.q), w.host(w.k_pool), w.host(w.v_pool), w.block_tables, c, w.scale,
+                                   B, "bf16") for i, c in enumerate(ctx_sets)}
+    for k, ((c, pt), out) in enumerate(zip(calls, outs)):
+        got = out.cpu().numpy()
+        assert np.all(np.isfinite(got)), (k, pt)
+        assert max_err(got, want[k % 3]) <= TOL["bf16"], (k, pt, max_err(got, want[k % 3]))
