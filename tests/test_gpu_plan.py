@@ -132,7 +132,8 @@ def test_back_to_back_calls_share_one_workspace(dev, H, Hq):
     rng = np.random.default_rng(1200 + Hq)
     ctx_sets = [rng.integers(0, mb * B + 1, S) for _ in range(3)]
     ctx_sets[1][:5] = 0
-    w = wl.build_paged(ctx_sets[0], H=H, D=128, B=B, dtype="bf16", seed=1201 + Hq, device=dev, max_blocks=mb,
+    # tables and pool cover the longest of the three lengths of every sequence
+    w = wl.build_paged(np.maximum.reduce(ctx_sets), H=H, D=128, B=B, dtype="bf16", seed=1201 + Hq, device=dev, max_blocks=mb,
                        num_q_heads=Hq)
     ix = dev_indices(w, dev)
     ws = pkv.alloc_workspace(w.q, w.k_pool, ix["bt"], 64)  # the largest of the plans below
