@@ -22,8 +22,8 @@ import numpy as np
 
 # paged_attn_decode on one B200 (batch-256 OPT-13B layer, bf16, contexts U[1,2048],
 # bench.py --block-size sweep, the attention call's roofline.achieved): effective
-# K/V GB/s per block size, measured with the two-stage-ring decode kernel.
-B200_DECODE_GBS = {8: 6922.0, 16: 7072.0, 32: 7148.0, 64: 7199.0, 128: 7209.0}
+# K/V GB/s per block size, measured with the current decode kernel (one sweep, one box).
+B200_DECODE_GBS = {8: 7186.0, 16: 7330.0, 32: 7392.0, 64: 7400.0, 128: 7447.0}
 
 
 def last_block_waste(context_lens, block_size):
