@@ -106,7 +106,7 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
 
 // Bulk (TMA-engine) copy of `bytes` contiguous bytes from global to this CTA's
 // shared memory; completion is reported to `bar` as transaction bytes.  Both
-// addresses 16-byte aligned, bytes a multiple of 16.  No cluster multicast.
+// addresses 16-byte aligned, bytes a multiple of 16.  The copy lands in this CTA only.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar,
                                           uint64_t policy) {
   asm volatile(
