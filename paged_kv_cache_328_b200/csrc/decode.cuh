@@ -93,6 +93,36 @@ __device__ __forceinline__ void fma_x2(float& d0, float& d1, float a0, float a1,
   asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
 }
 
+// d0 += a.lo * b.lo and d1 += a.hi * b.hi for two packed 16-bit pairs, accumulated in
+// fp32 (mixed-precision FMA, sm_100): the product of two 16-bit values is exact in fp32 and
+// each sum is rounded once, as fmaf on the widened values would be, with no widening step.
+template <typename T>
+struct MixedFma;
+template <>
+struct MixedFma<__nv_bfloat16> {
+  static __device__ __forceinline__ void pair(uint32_t a, uint32_t b, float& d0, float& d1) {
+    asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\t"
+        "mov.b32 {a0, a1}, %2;\n\t"
+        "mov.b32 {b0, b1}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, a0, b0, %0;\n\t"
+        "fma.rn.f32.bf16 %1, a1, b1, %1;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "r"(a), "r"(b));
+  }
+};
+template <>
+struct MixedFma<__half> {
+  static __device__ __forceinline__ void pair(uint32_t a, uint32_t b, float& d0, float& d1) {
+    asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\t"
+        "mov.b32 {a0, a1}, %2;\n\t"
+        "mov.b32 {b0, b1}, %3;\n\t"
+        "fma.rn.f32.f16 %0, a0, b0, %0;\n\t"
+        "fma.rn.f32.f16 %1, a1, b1, %1;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "r"(a), "r"(b));
+  }
+};
+
 struct DecodeParams {
   const void* q;
   const void* k_cache;
@@ -571,10 +601,16 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
   const int sub = lane & 7;   // which 16-byte chunks of a row this lane owns
   const int tok_lane = warp * 4 + grp;
 
-  float qf[Tr::kDimsPerLane];
+  constexpr bool kNarrow = sizeof(T) == 2;  // 16-bit storage: q stays packed, q.k in mixed precision
+  float qf[kNarrow ? 1 : Tr::kDimsPerLane];   // fp32 storage: q * scale_log2
+  uint4 qw[Tr::kChunksPerLane];               // 16-bit storage: this lane's chunks of q
   float acc[Tr::kDimsPerLane];
 #pragma unroll
-  for (int k = 0; k < Tr::kDimsPerLane; ++k) qf[k] = acc[k] = 0.f;
+  for (int k = 0; k < Tr::kDimsPerLane; ++k) acc[k] = 0.f;
+#pragma unroll
+  for (int k = 0; k < (kNarrow ? 1 : Tr::kDimsPerLane); ++k) qf[k] = 0.f;
+#pragma unroll
+  for (int c = 0; c < Tr::kChunksPerLane; ++c) qw[c] = make_uint4(0u, 0u, 0u, 0u);
   float m = -INFINITY, l = 0.f;
   int units_done = 0;
 
@@ -599,10 +635,15 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
       for (int k = 0; k < Tr::kDimsPerLane; ++k) acc[k] = 0.f;
       if (n_valid > 0) {
         const uint4* qrow = reinterpret_cast<const uint4*>(smem + Tr::kQOffset + stage * Tr::kRowBytes);
+        if constexpr (kNarrow) {
 #pragma unroll
-        for (int c = 0; c < Tr::kChunksPerLane; ++c) Elem<T>::widen(qrow[c * 8 + sub], qf + c * Tr::kPerChunk);
+          for (int c = 0; c < Tr::kChunksPerLane; ++c) qw[c] = qrow[c * 8 + sub];
+        } else {
 #pragma unroll
-        for (int k = 0; k < Tr::kDimsPerLane; ++k) qf[k] *= prm.scale_log2;
+          for (int c = 0; c < Tr::kChunksPerLane; ++c) Elem<T>::widen(qrow[c * 8 + sub], qf + c * Tr::kPerChunk);
+#pragma unroll
+          for (int k = 0; k < Tr::kDimsPerLane; ++k) qf[k] *= prm.scale_log2;
+        }
       }
     }
 
@@ -617,13 +658,17 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
         const uint4* row = reinterpret_cast<const uint4*>(kt + r * Tr::kRowBytes);
 #pragma unroll
         for (int c = 0; c < Tr::kChunksPerLane; ++c) {
-          float f[Tr::kPerChunk];
-          Elem<T>::widen(row[c * 8 + sub], f);
+          if constexpr (kNarrow) {
+            const uint4 kw = row[c * 8 + sub];
+            MixedFma<T>::pair(qw[c].x, kw.x, d0, d1);
+            MixedFma<T>::pair(qw[c].y, kw.y, d0, d1);
+            MixedFma<T>::pair(qw[c].z, kw.z, d0, d1);
+            MixedFma<T>::pair(qw[c].w, kw.w, d0, d1);
+          } else {
+            float f[Tr::kPerChunk];
+            Elem<T>::widen(row[c * 8 + sub], f);
 #pragma unroll
-          for (int k = 0; k < Tr::kPerChunk; k += 2) {
-            if constexpr (sizeof(T) == 2) {
-              fma_x2(d0, d1, qf[c * Tr::kPerChunk + k], qf[c * Tr::kPerChunk + k + 1], f[k], f[k + 1]);
-            } else {  // (fp32 storage: scalar, which keeps that instantiation free of spills)
+            for (int k = 0; k < Tr::kPerChunk; k += 2) {
               d0 = fmaf(qf[c * Tr::kPerChunk + k], f[k], d0);
               d1 = fmaf(qf[c * Tr::kPerChunk + k + 1], f[k + 1], d1);
             }
@@ -634,6 +679,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
       d += __shfl_xor_sync(0xffffffffu, d, 1);
       d += __shfl_xor_sync(0xffffffffu, d, 2);
       d += __shfl_xor_sync(0xffffffffu, d, 4);
+      if constexpr (kNarrow) d *= prm.scale_log2;  // (fp32 storage: q carries the scale)
       x[j] = (r < n_valid) ? d : -INFINITY;
     }
 
