@@ -688,7 +688,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
     for (int j = 1; j < Tr::kTokPerGroup; ++j) mt = fmaxf(mt, x[j]);
     const float m_new = fmaxf(m, mt);
     if (m_new != -INFINITY) {
-      const float alpha = exp2f(m - m_new);  // 0 while m is still -inf
+      const float alpha = ex2_fast(m - m_new);  // 0 while m is still -inf
       l *= alpha;
 #pragma unroll
       for (int k = 0; k < Tr::kDimsPerLane; ++k) acc[k] *= alpha;
@@ -696,7 +696,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
       for (int j = 0; j < Tr::kTokPerGroup; ++j) {
         const int r = j * Tr::kGroups + tok_lane;
         if (r < n_valid) {  // rows past the context are never read (they may hold NaN)
-          const float pj = exp2f(x[j] - m_new);
+          const float pj = ex2_fast(x[j] - m_new);
           l += pj;
           const uint4* row = reinterpret_cast<const uint4*>(vt + r * Tr::kRowBytes);
 #pragma unroll

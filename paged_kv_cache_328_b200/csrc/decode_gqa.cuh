@@ -163,14 +163,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// 2^x with the hardware approximation (one MUFU instruction; relative error
-// ~2^-22; -inf gives +0, flush-to-zero).
-__device__ __forceinline__ float ex2_fast(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // A unit as the producer sees it: (sequence, K/V head, 16-row tile, partition).
 struct GqaUnit {
   int s, kvh, rt, p, t_begin, t_end, n_parts, ctx;

@@ -104,6 +104,14 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
   return policy;
 }
 
+// 2^x with the hardware approximation (one MUFU instruction; relative error
+// ~2^-22; -inf gives +0, flush-to-zero).
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Bulk (TMA-engine) copy of `bytes` contiguous bytes from global to this CTA's
 // shared memory; completion is reported to `bar` as transaction bytes.  Both
 // addresses 16-byte aligned, bytes a multiple of 16.  The copy lands in this CTA only.
