@@ -115,6 +115,16 @@ struct KtTraits {
   static_assert(kSmemAlloc <= 227 * 1024, "shared memory per CTA");
 };
 
+// (d0, d1) += (a0, a1): two fp32 additions in one packed instruction (sm_100), each
+// rounded as a scalar addition.
+__device__ __forceinline__ void add_x2(float& d0, float& d1, float a0, float a1) {
+  uint64_t d, a;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(d0), "f"(d1));
+  asm("add.rn.f32x2 %0, %0, %1;" : "+l"(d) : "l"(a));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
+
 // Non-blocking test of a barrier phase (mbarrier.test_wait never suspends the thread).
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   uint32_t done;
@@ -839,11 +849,15 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
         // a row that some token sees has a finite m_r (visibility is a prefix of the partition)
 #pragma unroll
         for (int c = 0; c < NH / 4; ++c) {
+          // x * scale - m_r, two rows per packed fp32 FMA (each rounded as fmaf)
           const float4 m = mref4[c];
-          x[4 * c] = fmaf(x[4 * c], scale, -m.x);
-          x[4 * c + 1] = fmaf(x[4 * c + 1], scale, -m.y);
-          x[4 * c + 2] = fmaf(x[4 * c + 2], scale, -m.z);
-          x[4 * c + 3] = fmaf(x[4 * c + 3], scale, -m.w);
+          float t0 = -m.x, t1 = -m.y, t2 = -m.z, t3 = -m.w;
+          fma_x2(t0, t1, x[4 * c], x[4 * c + 1], scale, scale);
+          fma_x2(t2, t3, x[4 * c + 2], x[4 * c + 3], scale, scale);
+          x[4 * c] = t0;
+          x[4 * c + 1] = t1;
+          x[4 * c + 2] = t2;
+          x[4 * c + 3] = t3;
         }
         mask_hidden();
         float tmax = -INFINITY;
@@ -918,8 +932,7 @@ __global__ void __launch_bounds__(kKtThreads, 1) paged_gqa_tc_kernel(const __gri
             const int r = 8 * c + 2 * i;
             const float p0 = ex2_fast(x[r]);  // 2^-inf = 0
             const float p1 = ex2_fast(x[r + 1]);
-            lpart[r] += p0;
-            lpart[r + 1] += p1;
+            add_x2(lpart[r], lpart[r + 1], p0, p1);
             split_pair<T>(p0, p1, hi[i], lo[i]);
           }
           const int col = r0 + 8 * c;
