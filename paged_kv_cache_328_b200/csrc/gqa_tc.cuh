@@ -115,16 +115,6 @@ struct KtTraits {
   static_assert(kSmemAlloc <= 227 * 1024, "shared memory per CTA");
 };
 
-// (d0, d1) += (a0, a1): two fp32 additions in one packed instruction (sm_100), each
-// rounded as a scalar addition.
-__device__ __forceinline__ void add_x2(float& d0, float& d1, float a0, float a1) {
-  uint64_t d, a;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(d0), "f"(d1));
-  asm("add.rn.f32x2 %0, %0, %1;" : "+l"(d) : "l"(a));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
-}
-
 // Non-blocking test of a barrier phase (mbarrier.test_wait never suspends the thread).
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   uint32_t done;

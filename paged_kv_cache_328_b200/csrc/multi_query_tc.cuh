@@ -246,6 +246,25 @@ __device__ __forceinline__ void split_pair<__half>(float p0, float p1, uint32_t&
   lo = Mma16816<__half>::pack(p0 - f.x, p1 - f.y);
 }
 
+// (d0, d1) += (a0, a1): two fp32 additions in one packed instruction (sm_100), each
+// rounded as a scalar addition.
+__device__ __forceinline__ void add_x2(float& d0, float& d1, float a0, float a1) {
+  uint64_t d, a;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(d0), "f"(d1));
+  asm("add.rn.f32x2 %0, %0, %1;" : "+l"(d) : "l"(a));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
+
+// (d0, d1) *= (a0, a1): two fp32 multiplications in one packed instruction (sm_100).
+__device__ __forceinline__ void mul_x2(float& d0, float& d1, float a0, float a1) {
+  uint64_t d, a;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(d0), "f"(d1));
+  asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(d) : "l"(a));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
+
 struct TcUnit {
   int s, kvh, rt, p, t_begin, t_end, n_parts, ctx;
 };
@@ -656,9 +675,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
       const int n_ok = max(0, min(n_valid, limit - t0));  // columns [0, n_ok) are visible
       float mt = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kTcTile; ++c) {
-        x[c] = c < n_ok ? x[c] * prm.scale_log2 : -INFINITY;
+      for (int c = 0; c < kTcTile; c += 2) {
+        float s0 = x[c], s1 = x[c + 1];
+        mul_x2(s0, s1, prm.scale_log2, prm.scale_log2);  // two columns per packed multiply
+        x[c] = c < n_ok ? s0 : -INFINITY;
+        x[c + 1] = c + 1 < n_ok ? s1 : -INFINITY;
         mt = fmaxf(mt, x[c]);
+        mt = fmaxf(mt, x[c + 1]);
       }
 
       // P buffer j & 1 was last read by the P V product of tile j - 2
@@ -705,14 +728,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_multi_query_tc_kernel(con
       // P = 2^(x - m_ref) as high + low 16-bit parts, written to this row's tensor-memory
       // lane: packed pairs, tokens 2c and 2c + 1 in column c
       uint32_t hi[kTcTile / 2], lo[kTcTile / 2];
+      float l0 = 0.f, l1 = 0.f;  // row-sum partials of the even and odd tokens
 #pragma unroll
       for (int c2 = 0; c2 < kTcTile / 2; ++c2) {
         const int c = 2 * c2;
-        const float p0 = x[c] == -INFINITY ? 0.f : ex2_fast(x[c] - m_ref);
-        const float p1 = x[c + 1] == -INFINITY ? 0.f : ex2_fast(x[c + 1] - m_ref);
-        l += p0 + p1;
+        float t0 = x[c], t1 = x[c + 1];
+        add_x2(t0, t1, -m_ref, -m_ref);  // x - m_ref, two tokens per packed add
+        const float p0 = x[c] == -INFINITY ? 0.f : ex2_fast(t0);
+        const float p1 = x[c + 1] == -INFINITY ? 0.f : ex2_fast(t1);
+        add_x2(l0, l1, p0, p1);
         split_pair<T>(p0, p1, hi[c2], lo[c2]);
       }
+      l += l0 + l1;
       {
         const uint32_t pcol = trow + Tr::kPCol + (uint32_t)(sb * 64);
         tmem_st16(pcol, *reinterpret_cast<uint32_t(*)[16]>(hi));
